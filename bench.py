@@ -1,0 +1,406 @@
+#!/usr/bin/env python3
+"""Benchmark of the Ring Attention hot path on B200.
+
+One step = one fused ring forward (all partitions, ring order, causal skip,
+online-softmax fold, epilogue) over one batch of synthetic input of the
+chosen workload.  The JSON line reports causal-adjusted TFLOP/s, the
+roofline of the dominant kernel, the end-to-end number through the public
+API from pinned host buffers, the oracle's CPU throughput on a bounded
+sample, and the pass-Q decode leg (GB/s of KV cache read) that the metric
+also names.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2|3|5|1]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, same line
+
+N > 1 (torchrun): every rank runs an independent replica of the workload
+(different seed), no collective on the data path; value = work of all ranks
+divided by the slowest rank's time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from ring_context_parallelism_ra_b200 import ra  # noqa: E402
+from ring_context_parallelism_ra_b200.workloads import (decode_kv_bytes, make_workload_inputs,  # noqa: E402
+                                                        prefill_flops, workload)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20   # > 126 MB L2
+METRIC = "causal attn TFLOP/s & % BF16 peak (prefill ring); decode GB/s & % HBM peak"
+
+
+# ---------------------------------------------------------------- helpers --
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "ring_context_parallelism_ra_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel_key, files):
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_sha") != kernel_source_sha(files):
+        return None
+    return e
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.nv = None
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvml unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    if world != n_gpus and world > 1:
+        print(f"warning: --gpus {n_gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ cpu oracle --
+
+def oracle_sample(wl, budget_s, seed=0):
+    """Time the fp64 oracle on a bounded sample of query rows of the workload
+    (drawn on the CPU with the workload recipe).  Returns (TFLOP/s, cores,
+    description)."""
+    from oracle.attention import attention as oracle_attention  # test infrastructure
+    from ring_context_parallelism_ra_b200.workloads import make_qkv
+    cores = len(os.sched_getaffinity(0))
+    n = wl.n
+    # one head-pair of the workload at full length (K, V of one KV head)
+    q, k, v = make_qkv(1, 1, 1, n, n, wl.d_qk, wl.d_v, wl.torch_dtype, wl.seed + 77, wl.qk_mult)
+    rng = np.random.default_rng(seed)
+    done_rows, flops, t0 = 0, 0.0, time.perf_counter()
+    chunk = max(8, min(512, 2 ** 22 // n))
+    while time.perf_counter() - t0 < budget_s:
+        rows = np.sort(rng.integers(0, n, chunk))
+        oracle_attention(q, k, v, wl.scale, wl.causal, rows=rows)
+        vis = (rows + 1) if wl.causal else np.full(len(rows), n)
+        flops += float(2.0 * vis.sum() * (wl.d_qk + wl.d_v))
+        done_rows += len(rows)
+    dt = time.perf_counter() - t0
+    desc = (f"{done_rows} random query rows of one head at n={n} (full key range each, "
+            f"causal FLOPs counted per row), {dt:.1f} s")
+    return flops / dt / 1e12, cores, desc
+
+
+# ------------------------------------------------------------- our arm ----
+
+def run_ours(args, world, rank):
+    dev = torch.device("cuda")
+    wl = workload(args.workload)
+    peaks, peaks_kind = load_peaks()
+    flops = prefill_flops(wl)
+    ra.lib()
+
+    # each replica draws its own inputs (seed offset by rank)
+    q, k, v = make_workload_inputs(dataclasses.replace(wl, seed=wl.seed + 1000 * rank), device=dev)
+    out = torch.empty((wl.B, wl.Hq, wl.n, wl.d_v), device=dev, dtype=wl.torch_dtype)
+    lse = torch.empty((wl.B, wl.Hq, wl.n), device=dev, dtype=torch.float32)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ra.ring_forward(q, k, v, wl.P, wl.causal, wl.scale, out, lse)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert ra.get_status() == ra.RA_OK
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches0 = ra.launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.zero_()                     # L2 flush between timed steps (not timed)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = ra.launch_count() - launches0
+    assert ra.get_status() == ra.RA_OK
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_local = statistics.mean(per_step)
+    ms = max_over_ranks(ms_local, world)
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # roofline of the dominant (only) kernel of the step: one launch per step
+    kernel_files = ["simt_attention.cu"] if wl.dtype == "f32" else TC_FILES
+    achieved = flops / (ms_local * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tr = load_traffic(f"ring_forward:{wl.name}", kernel_files)
+    roofline = {"bound": "tensor" if wl.dtype == "bf16" else "alu", "achieved": round(achieved, 2),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                "peak_kind": f"{peaks_kind} bf16 burst", "kernel": "ring_forward",
+                "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", 1400.0), 4)}
+
+    # end to end through the public API from pinned host buffers
+    qh = q.cpu().pin_memory()
+    kh = k.cpu().pin_memory()
+    vh = v.cpu().pin_memory()
+    bufs = {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
+            "out": out, "lse": lse,
+            "out_h": torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
+            "lse_h": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)}
+    for _ in range(2):
+        ra.ring_forward_host(qh, kh, vh, wl.P, wl.causal, wl.scale, bufs=bufs)
+    e2e_steps = max(3, min(args.steps, 20))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        ra.ring_forward_host(qh, kh, vh, wl.P, wl.causal, wl.scale, bufs=bufs)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    e2e = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
+    del qh, kh, vh, bufs, q, k, v, out, lse, flush
+    torch.cuda.empty_cache()
+
+    decode = None if args.skip_decode else run_decode_leg(args, world, rank, peaks, peaks_kind)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "seq_len": wl.n,
+                   "d_qk": wl.d_qk, "d_v": wl.d_v, "P": wl.P, "causal": wl.causal,
+                   "flops_per_step": flops, "flop_convention": "2*B*Hq*n^2*(d_qk+d_v), x1/2 causal",
+                   "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if decode is not None:
+        line["decode"] = decode
+    return line
+
+
+TC_FILES = ["simt_attention.cu"]
+
+
+def run_decode_leg(args, world, rank, peaks, peaks_kind):
+    """Pass-Q decode over the 1M-token cache (P shards + merge): GB/s of K/V read."""
+    wl = workload(4)
+    dev = torch.device("cuda")
+    q, k, v = make_workload_inputs(wl, device=dev)
+    P = wl.P
+    L = wl.n // P
+    ws = torch.empty(ra.decode_workspace_bytes(wl.B, wl.Hq, wl.Hkv, L), dtype=torch.uint8, device=dev)
+    o_parts = torch.empty((P, wl.B, wl.Hq, wl.d_v), device=dev)
+    l_parts = torch.empty((P, wl.B, wl.Hq), device=dev)
+    out = torch.empty((wl.B, wl.Hq, wl.d_v), device=dev, dtype=wl.torch_dtype)
+    lse = torch.empty((wl.B, wl.Hq), device=dev)
+    bufs = {"o_parts": o_parts, "lse_parts": l_parts, "workspace": ws, "out": out, "lse": lse}
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        ra.decode_pass_q(q, k, v, P, wl.scale, bufs)
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 20))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for s, e in ev:
+            s.record(stream)
+            ra.decode_pass_q(q, k, v, P, wl.scale, bufs)
+            e.record(stream)
+        torch.cuda.synchronize()
+    assert ra.get_status() == ra.RA_OK
+    ms_local = statistics.mean(s.elapsed_time(e) for s, e in ev)
+    ms = max_over_ranks(ms_local, world)
+    nbytes = decode_kv_bytes(wl)
+    gbs = nbytes / (ms_local * 1e-3) / 1e9
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    del q, k, v, ws
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "value": round(world * nbytes / (ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s", "ms_per_step": round(ms, 4), "bytes_per_step": nbytes,
+            "launches_per_step": 2 * P + 1, "kv_bytes_exceed_l2": True,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "peak_kind": f"{peaks_kind} HBM copy",
+                         "kernel": "decode pass-Q (chunk kernel + two merges)"},
+            "clocks": clk.summary()}
+
+
+# -------------------------------------------------------- reference arm ----
+
+def run_reference(args, world, rank):
+    wl = workload(args.workload)
+    budget = float(os.environ.get("RA_ORACLE_BUDGET_S", "12"))
+    vals = []
+    desc, cores = "", 0
+    for i in range(args.warmup + args.steps):
+        per = budget / max(1, args.steps) if i >= args.warmup else min(2.0, budget / 10)
+        val, cores, desc = oracle_sample(wl, per, seed=i)
+        if i >= args.warmup:
+            vals.append(val)
+    value = statistics.mean(vals)
+    flops = prefill_flops(wl)
+    ms = flops / (value * 1e12) * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "seq_len": wl.n,
+                   "d_qk": wl.d_qk, "d_v": wl.d_v, "P": wl.P, "causal": wl.causal},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": desc + " per step"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 5])
+    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores only; other ranks do nothing
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if int(os.environ.get("RANK", "0")) == 0:
+            print(json.dumps(run_reference(args, world, 0)), flush=True)
+        return
+    world, rank, _ = dist_setup(args.gpus)
+    line = run_ours(args, world, rank)
+    if rank == 0:
+        val, cores, desc = oracle_sample(workload(args.workload), args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

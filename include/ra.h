@@ -1,0 +1,219 @@
+/*
+ * ra.h -- C ABI of the Ring Attention hot path on one B200 (sm_100a).
+ *
+ * What is computed (pages cited by title and section / equation):
+ *   O = softmax(scale * Q K^T + mask) V, exactly, per (batch, query head),
+ *   page "长上下文的第一性挑战", Eq. (lc-ch-attention).  The sequence is split
+ *   into P contiguous partitions; query partition i stays in place while the
+ *   KV partitions pass it in ring order (i, i-1, ..., i-P+1 mod P), page
+ *   "AI 推理系列（十一）：Ring Attention 如何让多张 GPU 共同计算一条超长序列",
+ *   section "KV 在 Ring 中如何流动".  Each (Q_i, KV_j) block is folded into a
+ *   running row max / exponential sum / rescaled output, never materialising
+ *   the n x n score matrix (same page, section "最容易被忽略的细节"), and blocks
+ *   wholly in the causal future are skipped.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major BHSD in device memory owned by the caller:
+ *       q    [B, Hq,  n_q, d_qk]     k [B, Hkv, n_k, d_qk]    v [B, Hkv, n_k, d_v]
+ *       out  [B, Hq,  n_q, d_v]      lse [B, Hq, n_q] (fp32, natural log,
+ *       scale included).  Grouped-query heads: query head h reads KV head
+ *       h / (Hq / Hkv).
+ *   - Causal rule: key at absolute position k_offset + u is visible to the
+ *     query at q_offset + t iff k_offset + u <= q_offset + t.
+ *   - Pointers must be 16-byte aligned.  The library allocates no device
+ *     memory per call; what it caches (TMA descriptors, a status word) is
+ *     created on first use and released by ra_shutdown().
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every
+ *     compute entry point only enqueues work and returns; it never
+ *     synchronises.  Results are ready when the stream reaches them.
+ *   - Return value: RA_OK or a negative ra_status.  Argument errors are found
+ *     on the host before anything is enqueued.  A device-side bounded wait
+ *     that expires cannot be returned by the launching call; it is recorded in
+ *     a per-device status word that ra_get_status() reads.
+ *   - Thread safety: calls may come from several host threads; the only
+ *     shared state (descriptor cache, status word) is guarded internally.
+ */
+#ifndef RA_H_
+#define RA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_INVALID = -1,      /* null / misaligned pointer, inconsistent shape   */
+  RA_ERR_UNSUPPORTED = -2,  /* valid request this build does not implement     */
+  RA_ERR_CUDA = -3,         /* a CUDA runtime call or kernel launch failed     */
+  RA_ERR_TIMEOUT = -4       /* a kernel's bounded wait expired (ra_get_status) */
+} ra_status;
+
+typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype;
+
+typedef struct {
+  int B;          /* batch                                                */
+  int Hq;         /* query heads                                          */
+  int Hkv;        /* KV heads; Hq % Hkv == 0                              */
+  int n_q;        /* query tokens per sequence                            */
+  int n_k;        /* key / value tokens per sequence (or per shard)       */
+  int d_qk;       /* head dim of Q and K                                  */
+  int d_v;        /* head dim of V and O                                  */
+  ra_dtype dtype; /* element type of q, k, v                              */
+} ra_shape;
+
+/*
+ * Supported head dims: bf16 d_qk in {64, 128, 192}, d_v in {64, 128} (tensor
+ * cores, tcgen05); fp32 d_qk, d_v in {64, 128} (exact fp32 FMA).
+ */
+
+/*
+ * ra_block_partial -- one (Q range, KV range) block: the partial of step a3 of
+ * the method, page "LLM长文本推理Ring Attention环形注意力机制实现与优化", section
+ * "Ring Attention实现代码与通信重叠" (each ring step computes the local
+ * attention of Q_i against the KV block that has arrived).
+ *   q, k, v     : device, BHSD as above (k, v hold the n_k keys of the block).
+ *   q_offset,
+ *   k_offset    : absolute position of the first query / key (causal mask).
+ *   causal      : 0 or 1.
+ *   scale       : multiplies Q K^T (normally 1/sqrt(d_qk)).
+ *   o_part      : device fp32 [B, Hq, n_q, d_v], normalised over this block's
+ *                 visible keys; a row with no visible key gets 0.
+ *   lse_part    : device fp32 [B, Hq, n_q]; -inf for a row with no visible key.
+ * Errors: RA_ERR_INVALID (null, misaligned, n <= 0, Hq % Hkv), RA_ERR_UNSUPPORTED
+ * (head dims), RA_ERR_CUDA (launch).
+ */
+int ra_block_partial(const void* q, const void* k, const void* v, const ra_shape* shape,
+                     int q_offset, int k_offset, int causal, float scale,
+                     float* o_part, float* lse_part, void* stream);
+
+/*
+ * ra_lse_merge -- N-way merge of normalised partials over disjoint key sets
+ * (step a6), the closed form of the beta / gamma update of page
+ * "LLM长文本推理Ring Attention环形注意力机制实现与优化", section
+ * "Ring Attention实现代码与通信重叠":
+ *   L* = max_p L_p,  w_p = exp(L_p - L*),  LSE = L* + ln sum w_p,
+ *   O = sum_p (w_p / sum w) O_p.   All L_p = -inf gives O = 0, LSE = -inf.
+ *   o_parts     : device fp32 [P, B, Hq, n_q, d_v] (P stacked partials).
+ *   lse_parts   : device fp32 [P, B, Hq, n_q].
+ *   shape       : B, Hq, n_q, d_v are read; dtype, Hkv, n_k, d_qk are ignored.
+ *   out         : device [B, Hq, n_q, d_v] of out_dtype (RA_F32 or RA_BF16).
+ *   lse         : device fp32 [B, Hq, n_q], or NULL to skip.
+ * Errors: RA_ERR_INVALID (P < 1, null, misaligned), RA_ERR_CUDA.
+ */
+int ra_lse_merge(const float* o_parts, const float* lse_parts, int P, const ra_shape* shape,
+                 void* out, ra_dtype out_dtype, float* lse, void* stream);
+
+/*
+ * ra_ring_forward -- the fused ring: all P partitions of one sequence in one
+ * kernel (steps a1-a5).  Query partition i meets KV partitions in ring order
+ * j = i, i-1, ..., i-P+1 (mod P); with causal = 1 the blocks j > i are
+ * skipped and the diagonal block is masked.  K/V tiles stream through a
+ * shared-memory ring filled by TMA while the previous tile's math runs.
+ *   q, k, v     : device BHSD, n_q == n_k == n, n % P == 0.
+ *   out         : device [B, Hq, n, d_v], same dtype as q.
+ *   lse         : device fp32 [B, Hq, n] (may be NULL).
+ * Errors: RA_ERR_INVALID (n_q != n_k, n % P, null, misaligned),
+ * RA_ERR_UNSUPPORTED (head dims), RA_ERR_CUDA.
+ */
+int ra_ring_forward(const void* q, const void* k, const void* v, int P, int causal, float scale,
+                    void* out, float* lse, const ra_shape* shape, void* stream);
+
+/*
+ * ra_decode_workspace_bytes -- bytes of device workspace ra_decode_partial
+ * needs for `shape` (its split-KV chunk partials).  0 on invalid shape.
+ */
+size_t ra_decode_workspace_bytes(const ra_shape* shape);
+
+/*
+ * ra_decode_partial -- pass-Q decode on one KV shard (step a7), page
+ * "上下文并行 (CP) 收益评估实验设计", decode section: the query is sent to every
+ * shard, each shard computes partial attention over its S/cp tokens, and the
+ * partials are reduced (ra_decode_merge).  One query token per sequence sees
+ * every token of the shard (no mask).
+ *   q           : device bf16 [B, Hq, 1, d_qk].
+ *   k_shard,
+ *   v_shard     : device bf16; head (b, g) of the shard starts at
+ *                 ptr + (b * Hkv + g) * kv_head_stride * d elements and holds
+ *                 n_k consecutive tokens (kv_head_stride = n_k for a dense
+ *                 shard, = the full cache length for a shard that is a token
+ *                 range of a larger [B, Hkv, S, d] cache).
+ *   shape       : n_q must be 1; n_k = shard length; d_qk == d_v == 128.
+ *   o_part      : device fp32 [B, Hq, d_v] normalised over the shard.
+ *   lse_part    : device fp32 [B, Hq].
+ *   workspace   : device, >= ra_decode_workspace_bytes(shape), 16-B aligned,
+ *                 owned by the caller; contents on entry are ignored.
+ * Errors: RA_ERR_INVALID, RA_ERR_UNSUPPORTED (dims, dtype), RA_ERR_CUDA.
+ */
+int ra_decode_partial(const void* q, const void* k_shard, const void* v_shard,
+                      long long kv_head_stride, const ra_shape* shape, float scale,
+                      float* o_part, float* lse_part, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
+ * ra_decode_merge -- reduce the P shard partials of pass-Q decode (step a8);
+ * the merge of ra_lse_merge with n_q = 1.
+ *   o_parts     : device fp32 [P, B, Hq, d_v];  lse_parts: [P, B, Hq].
+ *   out         : device [B, Hq, d_v] of out_dtype;  lse: fp32 [B, Hq] or NULL.
+ */
+int ra_decode_merge(const float* o_parts, const float* lse_parts, int P, const ra_shape* shape,
+                    void* out, ra_dtype out_dtype, float* lse, void* stream);
+
+/*
+ * ra_block_class -- causal class of every (query block, key block) pair,
+ * host side: 0 = SKIP (no visible pair), 1 = PARTIAL, 2 = FULL (every pair
+ * visible).  Blocks at the ragged end cover only existing rows / keys.  With
+ * causal = 0 every block is FULL.  This is the rule the kernels apply to their
+ * tiles (page "AI 推理系列（十一）…", section "KV 在 Ring 中如何流动": fully
+ * masked blocks may be skipped, the causal semantics must not change).
+ *   map_host    : host int8 [ceil(n_q/q_block), ceil(n_k/k_block)], row-major.
+ * Errors: RA_ERR_INVALID (null, non-positive sizes).
+ */
+int ra_block_class(int n_q, int n_k, int q_block, int k_block, int q_offset, int k_offset,
+                   int causal, int8_t* map_host);
+
+/*
+ * ra_block_class_device -- the same map computed by a kernel with the device
+ * copy of the rule the attention kernels use; map_dev is device memory.
+ */
+int ra_block_class_device(int n_q, int n_k, int q_block, int k_block, int q_offset,
+                          int k_offset, int causal, int8_t* map_dev, void* stream);
+
+/*
+ * ra_get_status -- synchronise `stream`, then read and clear the current
+ * device's status word.  Returns RA_OK, or RA_ERR_TIMEOUT if a kernel's
+ * bounded wait expired since the last call (its results are then invalid),
+ * or RA_ERR_CUDA if the synchronisation itself failed.
+ */
+int ra_get_status(void* stream);
+
+/*
+ * ra_set_wait_limit_ns -- bound, in nanoseconds, on every device-side wait of
+ * later launches (default 2e9).  Values below 1e6 are raised to 1e6.
+ */
+int ra_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * ra_check_wait_timeout -- launch one block whose wait nobody satisfies, so
+ * that its bounded wait runs out after `limit_ns`; the kernel records
+ * RA_ERR_TIMEOUT in the status word and returns normally.  Used to test the
+ * timeout path without faulting or hanging the GPU.
+ */
+int ra_check_wait_timeout(unsigned long long limit_ns, void* stream);
+
+/* Human-readable name of a status code. */
+const char* ra_status_string(int status);
+
+/* Number of kernel launches this library has enqueued since load. */
+unsigned long long ra_launch_count(void);
+
+/* Release cached descriptors.  Safe to call more than once. */
+int ra_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RA_H_ */

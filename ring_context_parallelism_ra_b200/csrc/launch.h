@@ -1,0 +1,50 @@
+// Host-side launchers of the kernels, called by the C ABI in ra_api.cu after
+// argument validation.  Each returns an ra_status.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ra.h"
+#include "common.cuh"
+
+namespace ra {
+
+// Counts kernel launches enqueued by this library (ra_launch_count).
+void note_launch();
+
+// Per-device state: SM count, status word address, wait bound.
+struct DeviceInfo {
+  int device;
+  int num_sms;
+  int max_smem_optin;
+  DevCtx ctx;
+};
+int device_info(DeviceInfo* out);
+
+int launch_lse_merge(const float* o_parts, const float* lse_parts, int P, long long rows, int d_v,
+                     void* out, ra_dtype out_dtype, float* lse, int num_sms, cudaStream_t stream);
+
+// Exact-fp32 (SIMT) attention: block partial (P = 1, offsets) or the fused
+// ring (P >= 1, offsets 0).  out_f32 selects fp32 output (partials).
+int launch_simt_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
+                          int q_offset, int k_offset, int causal, float scale, void* out,
+                          bool out_f32, float* lse, const DeviceInfo& dev, cudaStream_t stream);
+
+// Tensor-core (tcgen05) attention, bf16 inputs.
+int launch_tc_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
+                        int q_offset, int k_offset, int causal, float scale, void* out,
+                        bool out_f32, float* lse, const DeviceInfo& dev, cudaStream_t stream);
+
+// Decode: chunk partials of one shard into the workspace, then the merge.
+size_t decode_workspace_bytes(const ra_shape& s);
+int launch_decode_partial(const void* q, const void* k, const void* v, long long kv_head_stride,
+                          const ra_shape& s, float scale, float* o_part, float* lse_part,
+                          float* workspace, const DeviceInfo& dev, cudaStream_t stream);
+
+int launch_block_class(int n_q, int n_k, int q_block, int k_block, int q_offset, int k_offset,
+                       int causal, int8_t* map_dev, cudaStream_t stream);
+
+int launch_wait_timeout_check(const DevCtx& ctx, cudaStream_t stream);
+
+}  // namespace ra

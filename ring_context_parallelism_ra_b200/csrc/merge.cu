@@ -1,0 +1,98 @@
+// N-way LSE merge of normalised partials (O_p, L_p) over disjoint key sets.
+//
+//   L* = max_p L_p,  w_p = exp(L_p - L*),  LSE = L* + ln sum_p w_p,
+//   O  = sum_p (w_p / sum_q w_q) O_p
+//
+// This is the closed form of the beta / gamma fold of page "LLM长文本推理Ring
+// Attention环形注意力机制实现与优化", section "Ring Attention实现代码与通信重叠",
+// applied to P partials at once; partials with L_p = -inf carry no weight.
+//
+// HBM-bound: each output row reads P * (d_v + 1) floats once.  A row of d_v
+// floats is read as d_v / 4 float4 by d_v / 4 lanes (a warp covers one row at
+// d_v = 128, two at 64), with streaming loads since nothing is re-read.
+#include "common.cuh"
+#include "launch.h"
+
+namespace ra {
+
+template <typename OutT>
+__device__ __forceinline__ void store4(OutT* dst, float4 v);
+
+template <>
+__device__ __forceinline__ void store4<float>(float* dst, float4 v) {
+  *reinterpret_cast<float4*>(dst) = v;
+}
+
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4 v) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 packed;
+  packed.x = *reinterpret_cast<uint32_t*>(&lo);
+  packed.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(dst) = packed;
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ o_parts,
+                                                        const float* __restrict__ lse_parts,
+                                                        int P, long long rows, int d_v,
+                                                        OutT* __restrict__ out,
+                                                        float* __restrict__ lse_out) {
+  const int lanes_per_row = d_v >> 2;            // 32 (d_v = 128) or 16 (d_v = 64)
+  const int rows_per_warp = 32 / lanes_per_row;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / lanes_per_row;
+  const int col = (lane % lanes_per_row) * 4;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const long long part_stride = rows * d_v;
+
+  for (long long r = warp * rows_per_warp + sub; r < rows; r += n_warps * rows_per_warp) {
+    float m = -INFINITY;
+    for (int p = 0; p < P; ++p) m = fmaxf(m, __ldg(lse_parts + p * rows + r));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float w_sum = 0.f;
+    if (m != -INFINITY) {
+      const float* src = o_parts + r * d_v + col;
+#pragma unroll 4
+      for (int p = 0; p < P; ++p) {
+        const float l = __ldg(lse_parts + p * rows + r);
+        const float4 o = __ldcs(reinterpret_cast<const float4*>(src + p * part_stride));
+        const float w = (l == -INFINITY) ? 0.f : expf(l - m);
+        w_sum += w;
+        acc.x = fmaf(w, o.x, acc.x);
+        acc.y = fmaf(w, o.y, acc.y);
+        acc.z = fmaf(w, o.z, acc.z);
+        acc.w = fmaf(w, o.w, acc.w);
+      }
+      const float inv = 1.f / w_sum;
+      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+    }
+    store4<OutT>(out + r * d_v + col, acc);
+    if (lse_out != nullptr && col == 0) {
+      lse_out[r] = (m == -INFINITY) ? -INFINITY : m + logf(w_sum);
+    }
+  }
+}
+
+int launch_lse_merge(const float* o_parts, const float* lse_parts, int P, long long rows, int d_v,
+                     void* out, ra_dtype out_dtype, float* lse, int num_sms, cudaStream_t stream) {
+  const int threads = 256;
+  const int rows_per_cta = (threads / 32) * (32 / (d_v / 4));
+  long long want = (rows + rows_per_cta - 1) / rows_per_cta;
+  long long cap = static_cast<long long>(num_sms) * 8;   // 8 resident CTAs / SM
+  int grid = static_cast<int>(want < cap ? want : cap);
+  if (grid < 1) grid = 1;
+  if (out_dtype == RA_F32) {
+    lse_merge_kernel<float><<<grid, threads, 0, stream>>>(o_parts, lse_parts, P, rows, d_v,
+                                                          static_cast<float*>(out), lse);
+  } else {
+    lse_merge_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
+        o_parts, lse_parts, P, rows, d_v, static_cast<__nv_bfloat16*>(out), lse);
+  }
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+}  // namespace ra

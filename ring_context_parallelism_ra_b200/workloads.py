@@ -5,11 +5,14 @@ tests, the bench and the oracle side: it draws the inputs, and both the CUDA
 path and the fp64 oracle consume the same tensors.
 
 Recipe: every (tensor, batch, head) slice is drawn independently from
-``torch.Generator('cpu').manual_seed(seed)`` as i.i.d. N(0, 1) fp32, where the
+``torch.Generator(device).manual_seed(seed)`` as i.i.d. N(0, 1) fp32, where the
 seed is a fixed function of (workload seed, tensor, batch, head); Q and K are
 then multiplied by the workload's ``qk_mult`` (exact, a power of two) and the
-result is rounded to the workload dtype.  Drawing per head lets the oracle
-regenerate only the heads it samples.
+result is rounded to the workload dtype.  Large workloads are drawn directly
+on the GPU (torch's own generator; the CPU draws 10^8 values per second at
+best) and the oracle receives CPU copies of the slices it checks; small ones
+are drawn on the CPU.  The two devices give different (equally valid) values
+for the same seed, so one test never mixes them.
 
 The five workloads mirror the shapes the pages discuss: grouped-query heads
 with d = 128, 8K to 1M tokens, P = 4..16 partitions, an MLA-like head with
@@ -80,35 +83,35 @@ def _slice_seed(seed: int, tensor: str, b: int, h: int) -> int:
 
 
 def draw_slice(seed: int, tensor: str, b: int, h: int, rows: int, d: int,
-               dtype=torch.bfloat16, mult: float = 1.0) -> torch.Tensor:
-    """One [rows, d] slice on the CPU, N(0,1) fp32 * mult, rounded to dtype."""
-    g = torch.Generator(device="cpu").manual_seed(_slice_seed(seed, tensor, b, h))
-    x = torch.randn((rows, d), generator=g, dtype=torch.float32)
+               dtype=torch.bfloat16, mult: float = 1.0, device="cpu") -> torch.Tensor:
+    """One [rows, d] slice, N(0,1) fp32 * mult, rounded to dtype."""
+    g = torch.Generator(device=device).manual_seed(_slice_seed(seed, tensor, b, h))
+    x = torch.randn((rows, d), generator=g, dtype=torch.float32, device=device)
     if mult != 1.0:
         x.mul_(mult)
     return x.to(dtype)
 
 
 def make_qkv(B, Hq, Hkv, n_q, n_k, d_qk, d_v, dtype=torch.bfloat16, seed=0,
-             qk_mult=1.0, pin=False):
-    """Contiguous BHSD CPU tensors q [B,Hq,n_q,d_qk], k [B,Hkv,n_k,d_qk],
-    v [B,Hkv,n_k,d_v]."""
-    q = torch.empty((B, Hq, n_q, d_qk), dtype=dtype, pin_memory=pin)
-    k = torch.empty((B, Hkv, n_k, d_qk), dtype=dtype, pin_memory=pin)
-    v = torch.empty((B, Hkv, n_k, d_v), dtype=dtype, pin_memory=pin)
+             qk_mult=1.0, device="cpu"):
+    """Contiguous BHSD tensors q [B,Hq,n_q,d_qk], k [B,Hkv,n_k,d_qk],
+    v [B,Hkv,n_k,d_v] on `device`."""
+    q = torch.empty((B, Hq, n_q, d_qk), dtype=dtype, device=device)
+    k = torch.empty((B, Hkv, n_k, d_qk), dtype=dtype, device=device)
+    v = torch.empty((B, Hkv, n_k, d_v), dtype=dtype, device=device)
     for b in range(B):
         for h in range(Hq):
-            q[b, h] = draw_slice(seed, "q", b, h, n_q, d_qk, dtype, qk_mult)
+            q[b, h] = draw_slice(seed, "q", b, h, n_q, d_qk, dtype, qk_mult, device)
         for h in range(Hkv):
-            k[b, h] = draw_slice(seed, "k", b, h, n_k, d_qk, dtype, qk_mult)
-            v[b, h] = draw_slice(seed, "v", b, h, n_k, d_v, dtype)
+            k[b, h] = draw_slice(seed, "k", b, h, n_k, d_qk, dtype, qk_mult, device)
+            v[b, h] = draw_slice(seed, "v", b, h, n_k, d_v, dtype, 1.0, device)
     return q, k, v
 
 
-def make_workload_inputs(wl: Workload, pin=False):
-    """CPU tensors of a named workload (q has one row per sequence for decode)."""
+def make_workload_inputs(wl: Workload, device="cpu"):
+    """Tensors of a named workload (q has one row per sequence for decode)."""
     return make_qkv(wl.B, wl.Hq, wl.Hkv, wl.n_q, wl.n, wl.d_qk, wl.d_v,
-                    wl.torch_dtype, wl.seed, wl.qk_mult, pin=pin)
+                    wl.torch_dtype, wl.seed, wl.qk_mult, device=device)
 
 
 def prefill_flops(wl: Workload) -> float:

@@ -1,0 +1,46 @@
+"""Tolerances and comparison helpers for GPU-vs-oracle parity tests.
+
+Bars (stated for the method's outputs): bf16 inputs with fp32 accumulation
+give O within max-abs 2e-2 and mean-abs 2e-3 of the fp64 definition; fp32
+inputs give O within 1e-4; the log-sum-exp within 1e-3.
+"""
+import numpy as np
+import torch
+
+BF16_MAX_ABS = 2e-2
+BF16_MEAN_ABS = 2e-3
+F32_MAX_ABS = 1e-4
+LSE_MAX_ABS = 1e-3
+
+
+def to64(x):
+    if isinstance(x, torch.Tensor):
+        return x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def check_out(got, want, dtype, what="O"):
+    """Element-wise comparison of an output against the oracle."""
+    g, w = to64(got), to64(want)
+    assert g.shape == w.shape, (g.shape, w.shape)
+    assert np.isfinite(g).all(), f"{what}: non-finite values"
+    err = np.abs(g - w)
+    mx, mean = float(err.max()), float(err.mean())
+    if dtype in ("f32", torch.float32):
+        assert mx <= F32_MAX_ABS, f"{what}: max abs {mx:.3g} > {F32_MAX_ABS}"
+    else:
+        assert mx <= BF16_MAX_ABS, f"{what}: max abs {mx:.3g} > {BF16_MAX_ABS}"
+        assert mean <= BF16_MEAN_ABS, f"{what}: mean abs {mean:.3g} > {BF16_MEAN_ABS}"
+    return mx, mean
+
+
+def check_lse(got, want, what="LSE"):
+    g, w = to64(got), to64(want)
+    assert g.shape == w.shape, (g.shape, w.shape)
+    inf_g, inf_w = np.isneginf(g), np.isneginf(w)
+    assert np.array_equal(inf_g, inf_w), f"{what}: -inf pattern differs"
+    fin = ~inf_w
+    assert np.isfinite(g[fin]).all(), f"{what}: non-finite values"
+    mx = float(np.abs(g[fin] - w[fin]).max()) if fin.any() else 0.0
+    assert mx <= LSE_MAX_ABS, f"{what}: max abs {mx:.3g} > {LSE_MAX_ABS}"
+    return mx

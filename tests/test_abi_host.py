@@ -1,0 +1,104 @@
+"""CPU tests of the C ABI: the library loads, exports every symbol the header
+declares, and its host-side logic (argument validation, block classification)
+behaves, without launching anything on a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle.block_class import block_class as oracle_block_class
+from oracle.block_class import partition_class
+from ring_context_parallelism_ra_b200 import ra
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_symbols():
+    text = open(os.path.join(ROOT, "include", "ra.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ra_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = ra.lib()
+    syms = _header_symbols()
+    assert syms, "no declarations found in include/ra.h"
+    for name in syms:
+        assert hasattr(L, name), f"libra.so does not export {name}"
+    assert sorted(ra.EXPORTED) == syms
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4):
+        assert ra.status_string(code).startswith("RA_")
+    assert "unknown" in ra.status_string(7)
+
+
+@pytest.mark.parametrize("nq,nk,bq,bk", [(1, 1, 1, 1), (300, 300, 128, 128), (257, 511, 64, 128),
+                                         (1000, 200, 128, 64), (4096, 4096, 128, 128)])
+def test_host_block_class_matches_oracle(nq, nk, bq, bk):
+    for qo, ko in [(0, 0), (100, 0), (0, 77), (300, 299)]:
+        for causal in (0, 1):
+            got = ra.block_class(nq, nk, bq, bk, qo, ko, causal)
+            want = oracle_block_class(nq, nk, bq, bk, qo, ko, bool(causal))
+            np.testing.assert_array_equal(got, want)
+
+
+def test_host_partition_map_for_ring_configs():
+    for n, P in [(8192, 4), (131072, 8), (262144, 16)]:
+        got = ra.block_class(n, n, n // P, n // P, 0, 0, 1)
+        np.testing.assert_array_equal(got, partition_class(n, P, True))
+
+
+def _shape(**kw):
+    d = dict(B=1, Hq=2, Hkv=1, n_q=128, n_k=128, d_qk=128, d_v=128, dtype=ra.RA_BF16)
+    d.update(kw)
+    return ra.Shape(**d)
+
+
+def test_validation_rejects_bad_arguments_before_launch():
+    L = ra.lib()
+    p = ctypes.c_void_p(256)   # aligned dummy; never dereferenced on these paths
+    nul = ctypes.c_void_p(0)
+    mis = ctypes.c_void_p(258)
+    INV, UNS = ra.RA_ERR_INVALID, ra.RA_ERR_UNSUPPORTED
+    s = _shape()
+    assert L.ra_ring_forward(nul, p, p, 1, 1, 1.0, p, p, ctypes.byref(s), nul) == INV
+    assert L.ra_ring_forward(p, p, p, 0, 1, 1.0, p, p, ctypes.byref(s), nul) == INV
+    assert L.ra_ring_forward(p, p, p, 3, 1, 1.0, p, p, ctypes.byref(s), nul) == INV   # 128 % 3
+    assert L.ra_ring_forward(mis, p, p, 1, 1, 1.0, p, p, ctypes.byref(s), nul) == INV
+    s2 = _shape(n_k=64)
+    assert L.ra_ring_forward(p, p, p, 1, 1, 1.0, p, p, ctypes.byref(s2), nul) == INV  # n_q != n_k
+    s3 = _shape(Hq=3, Hkv=2)
+    assert L.ra_block_partial(p, p, p, ctypes.byref(s3), 0, 0, 1, 1.0, p, p, nul) == INV
+    s4 = _shape(d_qk=96)
+    assert L.ra_block_partial(p, p, p, ctypes.byref(s4), 0, 0, 1, 1.0, p, p, nul) == UNS
+    s5 = _shape(dtype=ra.RA_F32, d_qk=192)
+    assert L.ra_block_partial(p, p, p, ctypes.byref(s5), 0, 0, 1, 1.0, p, p, nul) == UNS
+    assert L.ra_block_partial(p, p, p, ctypes.byref(s), -1, 0, 1, 1.0, p, p, nul) == INV
+    assert L.ra_block_partial(p, p, p, ctypes.byref(s), 0, 0, 2, 1.0, p, p, nul) == INV
+    assert L.ra_block_partial(p, p, p, None, 0, 0, 1, 1.0, p, p, nul) == INV
+    assert L.ra_lse_merge(p, p, 0, ctypes.byref(s), p, 0, p, nul) == INV
+    s6 = _shape(d_v=96)
+    assert L.ra_lse_merge(p, p, 2, ctypes.byref(s6), p, 0, p, nul) == UNS
+    sd = _shape(n_q=1, Hq=8, Hkv=1, n_k=4096)
+    assert L.ra_decode_partial(p, p, p, 4096, ctypes.byref(sd), 1.0, p, p, p, 0, nul) == INV  # ws
+    assert L.ra_decode_partial(p, p, p, 100, ctypes.byref(sd), 1.0, p, p, p, 1 << 30, nul) == INV
+    sd2 = _shape(n_q=2, Hq=8, Hkv=1, n_k=4096)
+    assert L.ra_decode_partial(p, p, p, 4096, ctypes.byref(sd2), 1.0, p, p, p, 1 << 30, nul) == INV
+    sd3 = _shape(n_q=1, Hq=8, Hkv=1, n_k=4096, d_qk=64, d_v=64)
+    assert L.ra_decode_partial(p, p, p, 4096, ctypes.byref(sd3), 1.0, p, p, p, 1 << 30, nul) == UNS
+    assert L.ra_decode_merge(p, p, 2, ctypes.byref(_shape(n_q=4)), p, 0, p, nul) == INV
+    out = np.empty(4, dtype=np.int8)
+    assert L.ra_block_class(0, 4, 1, 1, 0, 0, 1, out.ctypes.data_as(ctypes.c_void_p)) == INV
+    assert L.ra_block_class(4, 4, 0, 1, 0, 0, 1, out.ctypes.data_as(ctypes.c_void_p)) == INV
+    assert L.ra_block_class(4, 4, 1, 1, 0, 0, 1, None) == INV
+
+
+def test_decode_workspace_size_is_chunk_partials():
+    # (chunks of 2048 tokens) x rows x (d + 1) floats, plus slack
+    n = ra.decode_workspace_bytes(4, 64, 8, 131072)
+    assert n >= 64 * 4 * 64 * 129 * 4
+    assert n < 64 * 4 * 64 * 129 * 4 + 4096

@@ -1,0 +1,85 @@
+"""GPU parity at the full workload sizes, in the launch configuration the bench
+times.  The oracle checks sampled outputs one by one (rows are independent,
+so each sampled row is an exact check); every other output is checked for
+finiteness.  Inputs are drawn on the GPU (see workloads.py) and the oracle
+receives CPU copies of the slices it needs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.attention import attention as oracle_attention
+from ring_context_parallelism_ra_b200 import ra
+from ring_context_parallelism_ra_b200.workloads import make_workload_inputs, workload
+from tests.parity_util import check_lse, check_out
+
+pytestmark = pytest.mark.gpu
+
+
+def sample_rows(n, P, tile=128, n_uniform=64, seed=0):
+    """Rows 0, 1, n-1; first/last row of every partition; first/last row of
+    the first and last four 128-row tiles of partitions 0 and P-1; plus
+    seeded uniform rows."""
+    L = n // P
+    rows = {0, 1, n - 1}
+    for i in range(P):
+        rows |= {i * L, i * L + L - 1}
+    for i in (0, P - 1):
+        nt = L // tile
+        for t in list(range(min(4, nt))) + list(range(max(0, nt - 4), nt)):
+            rows |= {i * L + t * tile, i * L + t * tile + tile - 1}
+    rng = np.random.default_rng(seed)
+    rows |= set(rng.integers(0, n, n_uniform).tolist())
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def _check_prefill(key, heads):
+    wl = workload(key)
+    torch.cuda.empty_cache()
+    q, k, v = make_workload_inputs(wl, device="cuda")
+    out, lse = ra.ring_forward(q, k, v, wl.P, wl.causal, wl.scale)
+    assert ra.get_status() == ra.RA_OK
+    assert torch.isfinite(out).all().item()
+    assert torch.isfinite(lse).all().item()
+    rows = sample_rows(wl.n, wl.P, seed=key)
+    G = wl.Hq // wl.Hkv
+    q_s = q[:, heads].cpu()
+    k_s = torch.stack([k[:, h // G] for h in heads], dim=1).cpu()
+    v_s = torch.stack([v[:, h // G] for h in heads], dim=1).cpu()
+    want_o, want_l = oracle_attention(q_s, k_s, v_s, wl.scale, wl.causal, rows=rows)
+    idx = torch.as_tensor(rows, device="cuda")
+    got_o = out[:, heads][:, :, idx]
+    got_l = lse[:, heads][:, :, idx]
+    check_out(got_o, want_o, wl.dtype)
+    check_lse(got_l, want_l)
+    del q, k, v, out, lse
+    torch.cuda.empty_cache()
+
+
+def test_config3_causal_gqa_128k():
+    _check_prefill(3, heads=[0, 3, 4, 31])
+
+
+def test_config5_causal_mla_256k():
+    _check_prefill(5, heads=[0, 15])
+
+
+def test_config4_decode_pass_q_1m():
+    wl = workload(4)
+    torch.cuda.empty_cache()
+    q, k, v = make_workload_inputs(wl, device="cuda")
+    out, lse = ra.decode_pass_q(q, k, v, wl.P, wl.scale)
+    assert ra.get_status() == ra.RA_OK
+    assert torch.isfinite(out).all().item() and torch.isfinite(lse).all().item()
+    G = wl.Hq // wl.Hkv
+    for b, g in [(0, 0), (3, 7), (1, 4)]:
+        heads = list(range(g * G, (g + 1) * G))
+        q_s = q[b:b + 1, heads].cpu()
+        k_s = k[b:b + 1, g:g + 1].cpu()
+        v_s = v[b:b + 1, g:g + 1].cpu()
+        want_o, want_l = oracle_attention(q_s, k_s, v_s, wl.scale, False)
+        check_out(out[b:b + 1, heads], want_o[:, :, 0], wl.dtype, f"O b={b} g={g}")
+        check_lse(lse[b:b + 1, heads], want_l[:, :, 0], f"LSE b={b} g={g}")
+    del q, k, v
+    torch.cuda.empty_cache()
