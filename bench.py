@@ -295,7 +295,7 @@ def run_ours(args, world, rank):
     return line
 
 
-TC_FILES = ["simt_attention.cu"]
+TC_FILES = ["tc_attention.cu", "ptx.cuh", "block_class.cuh"]
 
 
 def run_decode_leg(args, world, rank, peaks, peaks_kind):

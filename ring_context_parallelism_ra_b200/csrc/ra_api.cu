@@ -53,6 +53,9 @@ int dispatch_attention(const void* q, const void* k, const void* v, const ra_sha
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc != RA_OK) return rc;
+  if (s.dtype == RA_BF16)
+    return launch_tc_attention(q, k, v, s, P, q_offset, k_offset, causal, scale, out, out_f32,
+                               lse, dev, st);
   return launch_simt_attention(q, k, v, s, P, q_offset, k_offset, causal, scale, out, out_f32,
                                lse, dev, st);
 }

@@ -1,0 +1,578 @@
+// Tensor-core (tcgen05) attention for bf16 inputs: the fused ring forward and
+// the single-block partial.
+//
+// Method (pages cited by title and section): query partition i stays in place
+// while the KV partitions pass in ring order j = i, i-1, ..., i-P+1 (mod P)
+// ("AI 推理系列（十一）：Ring Attention 如何让多张 GPU 共同计算一条超长序列",
+// "KV 在 Ring 中如何流动"); a KV block wholly in the causal future is skipped
+// (same section); each visible block is folded into a running row max, a
+// running exponential sum and a rescaled output (same page, "最容易被忽略的细
+// 节"), never writing the score matrix to memory.  On one GPU the ring is a
+// schedule: the "next KV block" is the next K/V tile, prefetched by TMA into a
+// shared-memory ring while the tensor cores work on the current one (the
+// overlap of "通信很多，为什么仍然可能划算").
+//
+// CTA layout (320 threads, one CTA per SM, persistent):
+//   warps 0-3  softmax for query tile 0 (row r of the tile = thread r)
+//   warps 4-7  softmax for query tile 1
+//   warp 8     TMA producer: Q tiles, then K_j, V_j into a slot ring
+//   warp 9     tcgen05.mma issuer; owns the tensor-memory allocation
+// Work item = 256 query rows (two 128-row tiles) of one (batch, head); items
+// are dealt heaviest first in snake order across the persistent CTAs.
+//
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   [  0,128) S0 = Q0 K^T   (P0 as packed bf16 over its first 64 columns)
+//   [128,256) S1 = Q1 K^T   (P1 likewise)
+//   [256,256+DV) O0, [384,384+DV) O1   accumulators of P V
+// MMA issue order per KV tile j: PV0(j), S0(j+1), PV1(j), S1(j+1), so the
+// softmax of one tile overlaps the tensor-core work of the other.  MMAs from
+// one thread execute in issue order, so S_a(j+1) overwrites P_a(j) only after
+// PV_a(j) has read it, and a completed S_a(j+1) implies PV_a(j) is complete
+// (the softmax may then rescale O_a safely before releasing P_a(j+1)).
+// Rescaling is skipped unless the row max grows by more than 2^8 (the stale
+// max keeps p <= 256; the final division by l makes the result exact).
+#include <cuda.h>
+
+#include "block_class.cuh"
+#include "common.cuh"
+#include "launch.h"
+#include "ptx.cuh"
+#include "tmap.h"
+
+namespace ra {
+
+namespace {
+
+constexpr int kBM = 128;          // query rows per tile
+constexpr int kBN = 128;          // keys per KV tile
+constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16 = 16 KB
+constexpr int kThreads = 320;
+constexpr int kSmemLimit = 232448;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int DQK, int DV>
+struct Cfg {
+  static constexpr int QBOX = DQK / 64;
+  static constexpr int VBOX = DV / 64;
+  static constexpr int QTILE = QBOX * kBox;
+  static constexpr int SLOT = (QBOX > VBOX ? QBOX : VBOX) * kBox;
+  static constexpr int NSLOT_FIT = (kSmemLimit - 2048 - 2 * QTILE) / SLOT;
+  static constexpr int NSLOT = NSLOT_FIT > 6 ? 6 : NSLOT_FIT;
+  static constexpr int SMEM = 1024 + 2 * QTILE + NSLOT * SLOT + 1024;
+  static_assert(NSLOT >= 2, "need at least two K/V slots");
+  static_assert(SMEM <= kSmemLimit, "shared memory budget");
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, kBN, 0, 0);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, DV, 0, 1);
+};
+
+struct TcArgs {
+  int B, Hq, Hkv, n_q, n_k, P;
+  int q_offset, k_offset, causal;
+  float scale_log2;
+  void* out;          // [B*Hq, n_q, DV] bf16 or fp32
+  float* lse;         // [B*Hq, n_q] or null
+  int n_pairs, items;
+  DevCtx ctx;
+};
+
+// Query rows / ring partition of one work item.
+struct Item {
+  int bh, b, g;
+  int q0[2], qlen[2];
+  int i;  // ring partition of the item's first row
+};
+
+__device__ __forceinline__ bool item_at(const TcArgs& a, int round, Item& it) {
+  const int G = gridDim.x;
+  const int c = blockIdx.x;
+  const long long idx = static_cast<long long>(round) * G + ((round & 1) ? (G - 1 - c) : c);
+  if (idx >= a.items) return false;
+  const int bhs = a.B * a.Hq;
+  const int r = static_cast<int>(idx / bhs);
+  it.bh = static_cast<int>(idx % bhs);
+  const int tp = a.causal ? (a.n_pairs - 1 - r) : r;  // heaviest pairs first when causal
+  it.b = it.bh / a.Hq;
+  it.g = (it.bh % a.Hq) / (a.Hq / a.Hkv);
+  for (int t = 0; t < 2; ++t) {
+    it.q0[t] = tp * 2 * kBM + t * kBM;
+    const int rem = a.n_q - it.q0[t];
+    it.qlen[t] = rem <= 0 ? 0 : (rem < kBM ? rem : kBM);
+  }
+  const int Lq = a.n_q / a.P;
+  const int i = it.q0[0] / Lq;
+  it.i = i < a.P - 1 ? i : a.P - 1;
+  return true;
+}
+
+// The KV tiles an item visits, in ring order; every role runs this same walk.
+struct TileWalk {
+  int s, kt, kend;
+  __device__ __forceinline__ void start(const TcArgs& a, const Item& it) {
+    const int Lk = a.n_k / a.P;
+    s = 0;
+    kt = it.i * Lk;
+    kend = kt + Lk;
+  }
+  // Next tile with at least one active query tile: kt0, klen, class per tile.
+  __device__ __forceinline__ bool next(const TcArgs& a, const Item& it, int& kt0, int& klen,
+                                       int8_t (&cls)[2]) {
+    const int Lk = a.n_k / a.P;
+    while (true) {
+      if (kt >= kend) {
+        if (++s >= a.P) return false;
+        const int j = (it.i - s + a.P) % a.P;
+        kt = j * Lk;
+        kend = kt + Lk;
+        continue;
+      }
+      const int len = kend - kt < kBN ? kend - kt : kBN;
+      for (int t = 0; t < 2; ++t)
+        cls[t] = it.qlen[t] > 0 ? tile_class(it.q0[t], it.qlen[t], kt, len, a.q_offset,
+                                              a.k_offset, a.causal)
+                                : static_cast<int8_t>(kSkip);
+      if (cls[0] == kSkip && cls[1] == kSkip) {
+        // keys only grow inside a partition: with a causal mask nothing
+        // later in this partition is visible either
+        if (a.causal) kt = kend; else kt += kBN;
+        continue;
+      }
+      kt0 = kt;
+      klen = len;
+      kt += kBN;
+      return true;
+    }
+  }
+};
+
+template <int DQK, int DV>
+__device__ __forceinline__ void issue_s(uint32_t tmem_d, uint32_t q_base, uint32_t k_base) {
+#pragma unroll
+  for (int ks = 0; ks < DQK / 16; ++ks) {
+    const uint32_t off = (ks >> 2) * kBox + (ks & 3) * 32;
+    umma_ss(tmem_d, sdesc_k_sw128(q_base + off), sdesc_k_sw128(k_base + off), Cfg<DQK, DV>::IDESC_S,
+            ks > 0 ? 1u : 0u);
+  }
+}
+
+template <int DQK, int DV>
+__device__ __forceinline__ void issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_base,
+                                         bool accumulate) {
+#pragma unroll
+  for (int ks = 0; ks < kBN / 16; ++ks) {
+    umma_ts(tmem_d, tmem_p + ks * 8, sdesc_mn_sw128(v_base + ks * 2048, kBox),
+            Cfg<DQK, DV>::IDESC_PV, (accumulate || ks > 0) ? 1u : 0u);
+  }
+}
+
+template <int DQK, int DV, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, TcArgs a) {
+  using C = Cfg<DQK, DV>;
+  constexpr int NSLOT = C::NSLOT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = sm;
+  uint8_t* sKV = sm + 2 * C::QTILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NSLOT * C::SLOT);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* slot_full = bars + 2;
+  uint64_t* slot_empty = slot_full + NSLOT;
+  uint64_t* s_full = slot_empty + NSLOT;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* drain = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* kv_issued = abort_flag + 1;
+  volatile int* q_issued = abort_flag + 2;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(&slot_full[s], 1);
+      mbar_init(&slot_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], kBM);
+      mbar_init(&o_full[t], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *kv_issued = 0;
+    *q_issued = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      uint32_t ld = 0, qi = 0;
+      Item it;
+      for (int round = 0; !*abort_flag && item_at(a, round, it); ++round) {
+        if (!mbar_wait(q_empty, (qi & 1) ^ 1, a.ctx, abort_flag)) break;
+        mbar_arrive_expect_tx(q_full, 2 * C::QTILE);
+        for (int t = 0; t < 2; ++t)
+          for (int bx = 0; bx < C::QBOX; ++bx)
+            tma_load_3d(sQ + t * C::QTILE + bx * kBox, &tm_q, q_full, bx * 64, it.q0[t], it.bh);
+        *q_issued = static_cast<int>(++qi);
+        const int bkv = it.b * a.Hkv + it.g;
+        TileWalk w;
+        w.start(a, it);
+        int kt, klen;
+        int8_t cls[2];
+        bool ok = true;
+        while (ok && w.next(a, it, kt, klen, cls)) {
+          for (int part = 0; part < 2 && ok; ++part) {  // K then V
+            const int s = ld % NSLOT;
+            if (!mbar_wait(&slot_empty[s], ((ld / NSLOT) & 1) ^ 1, a.ctx, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint8_t* dst = sKV + s * C::SLOT;
+            if (part == 0) {
+              mbar_arrive_expect_tx(&slot_full[s], C::QBOX * kBox);
+              for (int bx = 0; bx < C::QBOX; ++bx)
+                tma_load_3d(dst + bx * kBox, &tm_k, &slot_full[s], bx * 64, kt, bkv);
+            } else {
+              mbar_arrive_expect_tx(&slot_full[s], C::VBOX * kBox);
+              for (int bx = 0; bx < C::VBOX; ++bx)
+                tma_load_3d(dst + bx * kBox, &tm_v, &slot_full[s], bx * 64, kt, bkv);
+            }
+            *kv_issued = static_cast<int>(++ld);
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      uint32_t ld = 0, qi = 0, pph[2] = {0, 0};
+      const uint32_t q_base[2] = {smem_u32(sQ), smem_u32(sQ + C::QTILE)};
+      const uint32_t kv_base = smem_u32(sKV);
+      Item it;
+      bool ok = true;
+      for (int round = 0; ok && item_at(a, round, it); ++round) {
+        if (!(ok = mbar_wait(q_full, qi & 1, a.ctx, abort_flag))) break;
+        ++qi;
+        tc_fence_after();
+        TileWalk w;
+        w.start(a, it);
+        int kt, klen;
+        int8_t cls[2], ncls[2];
+        bool any[2] = {false, false};
+        if (w.next(a, it, kt, klen, cls)) {
+          uint32_t kslot = ld % NSLOT, kph = (ld / NSLOT) & 1;
+          uint32_t vslot = (ld + 1) % NSLOT, vph = ((ld + 1) / NSLOT) & 1;
+          ld += 2;
+          if (!(ok = mbar_wait(&slot_full[kslot], kph, a.ctx, abort_flag))) break;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (cls[t] == kSkip) continue;
+            issue_s<DQK, DV>(tmem + t * 128, q_base[t], kv_base + kslot * C::SLOT);
+            umma_commit(&s_full[t]);
+          }
+          umma_commit(&slot_empty[kslot]);
+          while (true) {
+            int nkt, nklen;
+            const bool has_next = w.next(a, it, nkt, nklen, ncls);
+            uint32_t nkslot = 0, nkph = 0, nvslot = 0, nvph = 0;
+            if (has_next) {
+              nkslot = ld % NSLOT;
+              nkph = (ld / NSLOT) & 1;
+              nvslot = (ld + 1) % NSLOT;
+              nvph = ((ld + 1) / NSLOT) & 1;
+              ld += 2;
+            }
+            if (!(ok = mbar_wait(&slot_full[vslot], vph, a.ctx, abort_flag))) break;
+            tc_fence_after();
+            bool k_ready = false;
+            for (int t = 0; t < 2 && ok; ++t) {
+              if (cls[t] != kSkip) {
+                if (!(ok = mbar_wait(&p_full[t], pph[t] & 1, a.ctx, abort_flag))) break;
+                ++pph[t];
+                tc_fence_after();
+                issue_pv<DQK, DV>(tmem + 256 + t * 128, tmem + t * 128,
+                                  kv_base + vslot * C::SLOT, any[t]);
+                any[t] = true;
+              }
+              if (has_next && ncls[t] != kSkip) {
+                if (!k_ready) {
+                  if (!(ok = mbar_wait(&slot_full[nkslot], nkph, a.ctx, abort_flag))) break;
+                  tc_fence_after();
+                  k_ready = true;
+                }
+                issue_s<DQK, DV>(tmem + t * 128, q_base[t], kv_base + nkslot * C::SLOT);
+                umma_commit(&s_full[t]);
+              }
+            }
+            if (!ok) break;
+            umma_commit(&slot_empty[vslot]);
+            if (!has_next) break;
+            umma_commit(&slot_empty[nkslot]);
+            kslot = nkslot; kph = nkph; vslot = nvslot; vph = nvph;
+            kt = nkt; klen = nklen;
+            cls[0] = ncls[0];
+            cls[1] = ncls[1];
+          }
+          if (!ok) break;
+        }
+        for (int t = 0; t < 2; ++t)
+          if (any[t]) umma_commit(&o_full[t]);
+        umma_commit(q_empty);
+      }
+      // every MMA issued so far has finished before the allocation goes away
+      umma_commit(drain);
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < a.ctx.wait_ns) {
+      }
+    }
+  } else {
+    // ------------------------------------------------- softmax (2 x WG) --
+    const int t = warp >> 2;            // query tile of this warpgroup
+    const int row = threadIdx.x & 127;  // row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
+    const uint32_t s_col = t * 128;
+    const uint32_t o_col = 256 + t * 128;
+    uint32_t sph = 0, oph = 0;
+    Item it;
+    bool ok = true;
+    for (int round = 0; ok && item_at(a, round, it); ++round) {
+      float m = -INFINITY, l = 0.f;
+      bool any = false;
+      const long long q_pos = static_cast<long long>(a.q_offset) + it.q0[t] + row;
+      TileWalk w;
+      w.start(a, it);
+      int kt, klen;
+      int8_t cls[2];
+      while (w.next(a, it, kt, klen, cls)) {
+        if (cls[t] == kSkip) continue;
+        if (!(ok = mbar_wait(&s_full[t], sph & 1, a.ctx, abort_flag))) break;
+        ++sph;
+        tc_fence_after();
+        float s[kBN];
+        tmem_ld32f(lane_base + s_col, s);
+        tmem_ld32f(lane_base + s_col + 32, s + 32);
+        tmem_ld32f(lane_base + s_col + 64, s + 64);
+        tmem_ld32f(lane_base + s_col + 96, s + 96);
+        tmem_ld_wait();
+        reg_fence32(s);
+        reg_fence32(s + 32);
+        reg_fence32(s + 64);
+        reg_fence32(s + 96);
+        if (cls[t] == kPartial || klen < kBN) {
+          long long lim = klen;
+          if (a.causal) {
+            const long long vis = q_pos - (static_cast<long long>(a.k_offset) + kt) + 1;
+            lim = vis < lim ? vis : lim;
+          }
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+        const float m_cand = mx * a.scale_log2;
+        const bool grow = m_cand > m + kRescaleThreshold;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_cand);
+          m = m_cand;
+        }
+        const bool rescale_o = grow && l > 0.f;
+        l *= alpha;
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        float rs = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < kBN; c0 += 32) {
+          uint32_t p[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = fast_exp2(fmaf(s[c0 + c], a.scale_log2, neg_m));
+            const float p1 = fast_exp2(fmaf(s[c0 + c + 1], a.scale_log2, neg_m));
+            rs += p0 + p1;
+            p[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(lane_base + s_col + (c0 >> 1), p);
+        }
+        // O_a holds this item's sum only after its first PV; rescale it when a
+        // row of this warp needs it (tcgen05.ld/st are warp-collective).  The
+        // previous PV_a is complete: it was issued before S_a of this tile.
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          const float f = rescale_o ? alpha : 1.f;
+#pragma unroll
+          for (int c0 = 0; c0 < DV; c0 += 32) {
+            float o[32];
+            tmem_ld32f(lane_base + o_col + c0, o);
+            tmem_ld_wait();
+            reg_fence32(o);
+            uint32_t ob[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * f);
+            tmem_st32(lane_base + o_col + c0, ob);
+          }
+        }
+        tmem_st_wait();
+        l += rs;
+        any = true;
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l and LSE for the rows that exist ----
+      const bool valid = row < it.qlen[t];
+      const long long orow = static_cast<long long>(it.bh) * a.n_q + it.q0[t] + row;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      if (any) {
+        if (!(ok = mbar_wait(&o_full[t], oph & 1, a.ctx, abort_flag))) break;
+        ++oph;
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int c0 = 0; c0 < DV; c0 += 32) {
+        float o[32];
+        if (any) {
+          tmem_ld32f(lane_base + o_col + c0, o);
+          tmem_ld_wait();
+          reg_fence32(o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0.f;
+        }
+        if (valid) {
+          if constexpr (OUT_F32) {
+            float* dst = static_cast<float*>(a.out) + orow * DV + c0;
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(dst + c) =
+                  make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+          } else {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + orow * DV + c0;
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(o[c] * inv, o[c + 1] * inv);
+              v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
+              v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
+              v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
+              *reinterpret_cast<uint4*>(dst + c) = v;
+            }
+          }
+        }
+      }
+      if (valid && a.lse != nullptr)
+        a.lse[orow] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+      // the epilogue's TMEM reads are complete (wait::ld) before the next
+      // item's first P is released, so the next PV cannot overwrite O early
+    }
+  }
+
+  // ---------------------------------------------------------- teardown --
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_flag && threadIdx.x == 0) {
+    // let in-flight TMA loads land before shared memory is released (bounded)
+    const int n = *kv_issued;
+    for (int i = n - NSLOT < 0 ? 0 : n - NSLOT; i < n; ++i) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(&slot_full[i % NSLOT], (i / NSLOT) & 1) &&
+             globaltimer_ns() - t0 < a.ctx.wait_ns) {
+      }
+    }
+    const int nq = *q_issued;
+    if (nq > 0) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(q_full, (nq - 1) & 1) && globaltimer_ns() - t0 < a.ctx.wait_ns) {
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+template <int DQK, int DV, bool OUT_F32>
+int launch_typed(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const TcArgs& args, int grid, cudaStream_t stream) {
+  auto kern = tc_attention_kernel<DQK, DV, OUT_F32>;
+  constexpr int smem = Cfg<DQK, DV>::SMEM;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return RA_ERR_CUDA;
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, args);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+template <bool OUT_F32>
+int dispatch(int dqk, int dv, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+             const TcArgs& args, int grid, cudaStream_t st) {
+  if (dqk == 128 && dv == 128) return launch_typed<128, 128, OUT_F32>(tq, tk, tv, args, grid, st);
+  if (dqk == 192 && dv == 128) return launch_typed<192, 128, OUT_F32>(tq, tk, tv, args, grid, st);
+  if (dqk == 64 && dv == 64) return launch_typed<64, 64, OUT_F32>(tq, tk, tv, args, grid, st);
+  if (dqk == 64 && dv == 128) return launch_typed<64, 128, OUT_F32>(tq, tk, tv, args, grid, st);
+  if (dqk == 128 && dv == 64) return launch_typed<128, 64, OUT_F32>(tq, tk, tv, args, grid, st);
+  if (dqk == 192 && dv == 64) return launch_typed<192, 64, OUT_F32>(tq, tk, tv, args, grid, st);
+  return RA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+int launch_tc_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
+                        int q_offset, int k_offset, int causal, float scale, void* out,
+                        bool out_f32, float* lse, const DeviceInfo& dev, cudaStream_t stream) {
+  if (s.dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  const uint64_t hq = static_cast<uint64_t>(s.B) * s.Hq;
+  const uint64_t hkv = static_cast<uint64_t>(s.B) * s.Hkv;
+  if (make_tmap_bf16_3d(&tq, q, s.d_qk, s.n_q, hq, s.d_qk * 2ull,
+                        static_cast<uint64_t>(s.n_q) * s.d_qk * 2, 64, kBM) != 0 ||
+      make_tmap_bf16_3d(&tk, k, s.d_qk, s.n_k, hkv, s.d_qk * 2ull,
+                        static_cast<uint64_t>(s.n_k) * s.d_qk * 2, 64, kBN) != 0 ||
+      make_tmap_bf16_3d(&tv, v, s.d_v, s.n_k, hkv, s.d_v * 2ull,
+                        static_cast<uint64_t>(s.n_k) * s.d_v * 2, 64, kBN) != 0)
+    return RA_ERR_CUDA;
+  TcArgs a;
+  a.B = s.B;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.n_q = s.n_q;
+  a.n_k = s.n_k;
+  a.P = P;
+  a.q_offset = q_offset;
+  a.k_offset = k_offset;
+  a.causal = causal;
+  a.scale_log2 = scale * kLog2e;
+  a.out = out;
+  a.lse = lse;
+  a.n_pairs = (s.n_q + 2 * kBM - 1) / (2 * kBM);
+  const long long items = static_cast<long long>(a.n_pairs) * s.B * s.Hq;
+  if (items > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  a.items = static_cast<int>(items);
+  a.ctx = dev.ctx;
+  const int grid = a.items < dev.num_sms ? a.items : dev.num_sms;
+  return out_f32 ? dispatch<true>(s.d_qk, s.d_v, tq, tk, tv, a, grid, stream)
+                 : dispatch<false>(s.d_qk, s.d_v, tq, tk, tv, a, grid, stream);
+}
+
+}  // namespace ra
