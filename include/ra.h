@@ -153,6 +153,30 @@ int ra_decode_partial(const void* q, const void* k_shard, const void* v_shard,
                       void* stream);
 
 /*
+ * ra_decode_partial_noalloc -- ra_decode_partial without a caller workspace.
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot allocate device memory: a plugin inside a host runtime that owns all
+ * device memory and gives its plugins no allocator, or a latency-critical
+ * loop that must not call cudaMalloc (which may synchronise the device).
+ * The chunk partials live in one file-scope device array of 16 MiB, held on
+ * every GPU that loads the library until the process exits.  The call itself
+ * allocates nothing and calls no allocating routine.
+ *   Arguments, layout and results as ra_decode_partial, minus the workspace.
+ *   Limit: ceil(n_k / 2048) * B * Hq * (d_v + 1) * 4 + 256 bytes must not
+ *   exceed 16 MiB (e.g. a 131072-token shard with B * Hq = 256 needs 8.5 MB);
+ *   larger shapes return RA_ERR_UNSUPPORTED before anything is enqueued.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current) and caches it; make that first call before any
+ *   stream capture.  All calls share the array and it keeps the last call's
+ *   contents; calls whose kernels overlap on the GPU (e.g. on two unordered
+ *   streams) race on it, so order them on one stream.
+ * Errors: as ra_decode_partial.
+ */
+int ra_decode_partial_noalloc(const void* q, const void* k_shard, const void* v_shard,
+                              long long kv_head_stride, const ra_shape* shape, float scale,
+                              float* o_part, float* lse_part, void* stream);
+
+/*
  * ra_decode_merge -- reduce the P shard partials of pass-Q decode (step a8);
  * the merge of ra_lse_merge with n_q = 1.
  *   o_parts     : device fp32 [P, B, Hq, d_v];  lse_parts: [P, B, Hq].

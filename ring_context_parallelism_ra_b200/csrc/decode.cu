@@ -19,6 +19,8 @@
 // LSE merge) reduces the chunk partials to the shard partial.
 #include <cuda.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 #include "ptx.cuh"
@@ -362,6 +364,57 @@ int launch_decode_partial(const void* q, const void* k, const void* v, long long
   if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   return launch_lse_merge(a.ws_o, a.ws_lse, a.n_chunks, rows, kD, o_part, RA_F32, lse_part,
                           dev.num_sms, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  Some callers cannot allocate device memory: a
+// plugin inside a host runtime that owns all device memory and hands its
+// plugins no allocator, or a latency-critical loop that must not call
+// cudaMalloc (which may synchronise the device and has no latency bound).
+// For them the chunk partials live in this file-scope array instead of a
+// caller workspace.  Every GPU that loads the library holds the array until
+// the process exits.  Calls share it: two calls whose kernels overlap on the
+// GPU (different streams, no ordering between them) race on it.  Nothing in
+// it needs to start at zero, since the chunk kernel writes every partial that
+// the merge then reads; it keeps the last call's contents.
+constexpr size_t kStaticScratchBytes = 16u << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+namespace {
+
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[64] = {};
+
+// Device address of the scratch array for the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int scratch_address(int device, float** out) {
+  if (device < 0 || device >= 64) return RA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[device] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr)
+      return RA_ERR_CUDA;
+    g_scratch_ptr[device] = static_cast<float*>(p);
+  }
+  *out = g_scratch_ptr[device];
+  return RA_OK;
+}
+
+}  // namespace
+
+size_t decode_static_scratch_bytes() { return kStaticScratchBytes; }
+
+int launch_decode_partial_static(const void* q, const void* k, const void* v,
+                                 long long kv_head_stride, const ra_shape& s, float scale,
+                                 float* o_part, float* lse_part, const DeviceInfo& dev,
+                                 cudaStream_t stream) {
+  if (decode_workspace_bytes(s) > kStaticScratchBytes) return RA_ERR_UNSUPPORTED;
+  float* ws = nullptr;
+  const int rc = scratch_address(dev.device, &ws);
+  if (rc != RA_OK) return rc;
+  return launch_decode_partial(q, k, v, kv_head_stride, s, scale, o_part, lse_part, ws, dev,
+                               stream);
 }
 
 }  // namespace ra

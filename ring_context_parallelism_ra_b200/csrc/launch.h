@@ -42,6 +42,14 @@ int launch_decode_partial(const void* q, const void* k, const void* v, long long
                           const ra_shape& s, float scale, float* o_part, float* lse_part,
                           float* workspace, const DeviceInfo& dev, cudaStream_t stream);
 
+// Same without a caller workspace: the chunk partials go to a file-scope
+// device array of decode_static_scratch_bytes() bytes.
+size_t decode_static_scratch_bytes();
+int launch_decode_partial_static(const void* q, const void* k, const void* v,
+                                 long long kv_head_stride, const ra_shape& s, float scale,
+                                 float* o_part, float* lse_part, const DeviceInfo& dev,
+                                 cudaStream_t stream);
+
 int launch_block_class(int n_q, int n_k, int q_block, int k_block, int q_offset, int k_offset,
                        int causal, int8_t* map_dev, cudaStream_t stream);
 

@@ -214,6 +214,27 @@ int ra_decode_partial(const void* q, const void* k_shard, const void* v_shard,
                                static_cast<cudaStream_t>(stream));
 }
 
+int ra_decode_partial_noalloc(const void* q, const void* k_shard, const void* v_shard,
+                              long long kv_head_stride, const ra_shape* shape, float scale,
+                              float* o_part, float* lse_part, void* stream) {
+  int rc = check_common(shape);
+  if (rc != RA_OK) return rc;
+  if (!q || !k_shard || !v_shard || !o_part || !lse_part) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k_shard) || !aligned16(v_shard) || !aligned16(o_part) ||
+      !aligned16(lse_part))
+    return RA_ERR_INVALID;
+  if (shape->n_q != 1 || kv_head_stride < shape->n_k) return RA_ERR_INVALID;
+  if (shape->dtype != RA_BF16 || shape->d_qk != 128 || shape->d_v != 128 ||
+      shape->Hq / shape->Hkv > 16)
+    return RA_ERR_UNSUPPORTED;
+  if (decode_workspace_bytes(*shape) > decode_static_scratch_bytes()) return RA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc != RA_OK) return rc;
+  return launch_decode_partial_static(q, k_shard, v_shard, kv_head_stride, *shape, scale, o_part,
+                                      lse_part, dev, static_cast<cudaStream_t>(stream));
+}
+
 int ra_decode_merge(const float* o_parts, const float* lse_parts, int P, const ra_shape* shape,
                     void* out, ra_dtype out_dtype, float* lse, void* stream) {
   if (shape == nullptr || shape->n_q != 1) return RA_ERR_INVALID;

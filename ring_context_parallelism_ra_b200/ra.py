@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "RAError", "library_path", "lib", "Shape", "block_partial", "lse_merge", "ring_forward",
-    "ring_forward_host", "decode_workspace_bytes", "decode_partial", "decode_merge",
+    "ring_forward_host", "decode_workspace_bytes", "decode_partial", "decode_partial_noalloc",
+    "decode_merge",
     "decode_pass_q", "block_class", "block_class_device", "get_status", "set_wait_limit_ns",
     "check_wait_timeout", "launch_count", "status_string", "EXPORTED",
 ]
@@ -29,7 +30,7 @@ RA_F32, RA_BF16 = 0, 1
 # Every symbol include/ra.h declares.
 EXPORTED = (
     "ra_block_partial", "ra_lse_merge", "ra_ring_forward", "ra_decode_workspace_bytes",
-    "ra_decode_partial", "ra_decode_merge", "ra_block_class", "ra_block_class_device",
+    "ra_decode_partial", "ra_decode_partial_noalloc", "ra_decode_merge", "ra_block_class", "ra_block_class_device",
     "ra_get_status", "ra_set_wait_limit_ns", "ra_check_wait_timeout", "ra_status_string",
     "ra_launch_count", "ra_shutdown",
 )
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
             "ra_ring_forward": (i, [vp, vp, vp, i, i, f, vp, vp, sp, vp]),
             "ra_decode_workspace_bytes": (sz, [sp]),
             "ra_decode_partial": (i, [vp, vp, vp, ctypes.c_longlong, sp, f, vp, vp, vp, sz, vp]),
+            "ra_decode_partial_noalloc": (i, [vp, vp, vp, ctypes.c_longlong, sp, f, vp, vp, vp]),
             "ra_decode_merge": (i, [vp, vp, i, sp, vp, i, vp, vp]),
             "ra_block_class": (i, [i, i, i, i, i, i, i, vp]),
             "ra_block_class_device": (i, [i, i, i, i, i, i, i, vp, vp]),
@@ -241,6 +243,39 @@ def decode_partial(q, k, v, token_start=0, token_count=None, scale=None, workspa
                                  ctypes.c_size_t(workspace.numel() * workspace.element_size()),
                                  _stream(stream))
     _check("ra_decode_partial", rc)
+    return o_part, lse_part
+
+
+def decode_partial_noalloc(q, k, v, token_start=0, token_count=None, scale=None, o_part=None,
+                           lse_part=None, stream=None):
+    """decode_partial through ra_decode_partial_noalloc: the library keeps the
+    chunk partials in its own static device array, so no workspace is passed
+    (for callers that cannot allocate device memory).  Pass o_part / lse_part
+    to make the call itself allocation-free from Python as well."""
+    B, Hq, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence")
+    _, Hkv, S, dk = k.shape
+    token_count = S - token_start if token_count is None else token_count
+    if token_start < 0 or token_count <= 0 or token_start + token_count > S:
+        raise ValueError("shard outside the cache")
+    s = Shape(B, Hq, Hkv, 1, token_count, d, v.shape[-1], _dtype_code(q.dtype))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if o_part is None:
+        o_part = torch.empty((B, Hq, v.shape[-1]), device=q.device, dtype=torch.float32)
+    if lse_part is None:
+        lse_part = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    _need(k, "k", q.dtype)
+    _need(v, "v", q.dtype)
+    esz = k.element_size()
+    kp = ctypes.c_void_p(k.data_ptr() + token_start * dk * esz)
+    vp = ctypes.c_void_p(v.data_ptr() + token_start * v.shape[-1] * esz)
+    rc = lib().ra_decode_partial_noalloc(_need(q, "q"), kp, vp, ctypes.c_longlong(S),
+                                         ctypes.byref(s), float(scale),
+                                         _need(o_part, "o_part", torch.float32),
+                                         _need(lse_part, "lse_part", torch.float32),
+                                         _stream(stream))
+    _check("ra_decode_partial_noalloc", rc)
     return o_part, lse_part
 
 
