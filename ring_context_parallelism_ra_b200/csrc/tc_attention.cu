@@ -12,11 +12,19 @@
 // shared-memory ring while the tensor cores work on the current one (the
 // overlap of "通信很多，为什么仍然可能划算").
 //
-// CTA layout (320 threads, one CTA per SM, persistent):
+// CTA layout (384 threads, one CTA per SM, persistent):
 //   warps 0-3  softmax for query tile 0 (row r of the tile = thread r)
 //   warps 4-7  softmax for query tile 1
 //   warp 8     TMA producer: Q tiles, then K_j, V_j into a slot ring
 //   warp 9     tcgen05.mma issuer; owns the tensor-memory allocation
+//   warps 10-11 idle
+// Warp w runs on sub-partition w % 4, so each sub-partition holds one warp of
+// each warpgroup.  The kernel is launched with 168 registers per thread;
+// setmaxnreg then moves registers from the third warpgroup to the two softmax
+// warpgroups within that launch allocation: 2 x 208 + 88 = 504 = 3 x 168 per
+// lane.  (setmaxnreg.inc waits until registers are free, so a split above the
+// launch allocation would never proceed; the launcher checks the compiled
+// register count against the split before every launch.)
 // Work item = 256 query rows (two 128-row tiles) of one (batch, head); items
 // are dealt heaviest first in snake order across the persistent CTAs.
 //
@@ -46,7 +54,12 @@ namespace {
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per KV tile
 constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16 = 16 KB
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;    // per thread at launch (384 threads, 1 CTA / SM)
+constexpr int kRegsSoftmax = 208;   // per thread, softmax warpgroups
+constexpr int kRegsOther = 88;      // per thread, producer / MMA warpgroup
+static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kRegsLaunch,
+              "register split must fit the launch allocation");
 constexpr int kSmemLimit = 232448;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -144,23 +157,28 @@ struct TileWalk {
   }
 };
 
+// Descriptors of successive K steps differ only in the start-address field
+// (bits 0-13, address >> 4), which never carries out for shared memory, so
+// they are formed by adding (byte offset >> 4) to the tile's base descriptor.
 template <int DQK, int DV>
 __device__ __forceinline__ void issue_s(uint32_t tmem_d, uint32_t q_base, uint32_t k_base) {
+  const uint64_t da = sdesc_k_sw128(q_base);
+  const uint64_t db = sdesc_k_sw128(k_base);
 #pragma unroll
   for (int ks = 0; ks < DQK / 16; ++ks) {
-    const uint32_t off = (ks >> 2) * kBox + (ks & 3) * 32;
-    umma_ss(tmem_d, sdesc_k_sw128(q_base + off), sdesc_k_sw128(k_base + off), Cfg<DQK, DV>::IDESC_S,
-            ks > 0 ? 1u : 0u);
+    const uint32_t off = ((ks >> 2) * kBox + (ks & 3) * 32) >> 4;
+    umma_ss(tmem_d, da + off, db + off, Cfg<DQK, DV>::IDESC_S, ks > 0 ? 1u : 0u);
   }
 }
 
 template <int DQK, int DV>
 __device__ __forceinline__ void issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_base,
                                          bool accumulate) {
+  const uint64_t db = sdesc_mn_sw128(v_base, kBox);
 #pragma unroll
   for (int ks = 0; ks < kBN / 16; ++ks) {
-    umma_ts(tmem_d, tmem_p + ks * 8, sdesc_mn_sw128(v_base + ks * 2048, kBox),
-            Cfg<DQK, DV>::IDESC_PV, (accumulate || ks > 0) ? 1u : 0u);
+    umma_ts(tmem_d, tmem_p + ks * 8, db + ((ks * 2048) >> 4), Cfg<DQK, DV>::IDESC_PV,
+            (accumulate || ks > 0) ? 1u : 0u);
   }
 }
 
@@ -218,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) regs_dec<kRegsOther>();
   if (warp == 8) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
@@ -346,8 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < a.ctx.wait_ns) {
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------- softmax (2 x WG) --
+    regs_inc<kRegsSoftmax>();
     const int t = warp >> 2;            // query tile of this warpgroup
     const int row = threadIdx.x & 127;  // row within the tile = TMEM lane
     const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
@@ -389,9 +408,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
           for (int c = 0; c < kBN; ++c)
             if (c >= lim) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // row max: eight independent three-input max chains, then a tree
+        float mxs[8];
 #pragma unroll
-        for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+        for (int i = 0; i < 8; ++i) {
+          float v = fmax3(s[i], s[i + 8], s[i + 16]);
+#pragma unroll
+          for (int c = 24; c < 120; c += 16) v = fmax3(v, s[c + i], s[c + 8 + i]);
+          mxs[i] = fmaxf(v, s[120 + i]);
+        }
+        const float mx = fmax3(fmax3(mxs[0], mxs[1], mxs[2]), fmax3(mxs[3], mxs[4], mxs[5]),
+                               fmaxf(mxs[6], mxs[7]));
         const float m_cand = mx * a.scale_log2;
         const bool grow = m_cand > m + kRescaleThreshold;
         float alpha = 1.f;
@@ -402,19 +429,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
         const bool rescale_o = grow && l > 0.f;
         l *= alpha;
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
-        float rs = 0.f;
+        // p = 2^(s * scale_log2 - m): packed fp32x2 FMA, exp2, four packed
+        // partial sums, bf16 pairs stored into the P columns of tensor memory
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+        const float2 nm2 = make_float2(neg_m, neg_m);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c0 = 0; c0 < kBN; c0 += 32) {
           uint32_t p[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const float p0 = fast_exp2(fmaf(s[c0 + c], a.scale_log2, neg_m));
-            const float p1 = fast_exp2(fmaf(s[c0 + c + 1], a.scale_log2, neg_m));
-            rs += p0 + p1;
-            p[c >> 1] = pack_bf16x2(p0, p1);
+            const float2 x = __ffma2_rn(make_float2(s[c0 + c], s[c0 + c + 1]), sc2, nm2);
+            const float2 e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], e);
+            p[c >> 1] = pack_bf16x2(e.x, e.y);
           }
           tmem_st16(lane_base + s_col + (c0 >> 1), p);
         }
+        const float2 acc01 = __fadd2_rn(acc[0], acc[1]);
+        const float2 acc23 = __fadd2_rn(acc[2], acc[3]);
+        const float rs = (acc01.x + acc01.y) + (acc23.x + acc23.y);
         // O_a holds this item's sum only after its first PV; rescale it when a
         // row of this warp needs it (tcgen05.ld/st are warp-collective).  The
         // previous PV_a is complete: it was issued before S_a of this tile.
@@ -519,6 +554,7 @@ int launch_typed(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
   constexpr int smem = Cfg<DQK, DV>::SMEM;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return RA_ERR_CUDA;
+
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, args);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
