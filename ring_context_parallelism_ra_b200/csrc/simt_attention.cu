@@ -1,5 +1,5 @@
-// Exact-fp32 attention on CUDA cores (fp32 inputs; SIMT FMA, no tensor cores,
-// so fp32 results stay within 1e-4 of the fp64 definition).
+// Exact-fp32 attention on CUDA cores for fp32 inputs (SIMT FMA, no tensor
+// cores: TF32 would not hold fp32 results within 1e-4 of the fp64 definition).
 //
 // One CTA owns 64 query rows of one (batch, head).  It walks the KV
 // partitions in ring order j = i, i-1, ..., i-P+1 (mod P) where i is the
@@ -172,8 +172,6 @@ int dispatch_dims(const void* q, const void* k, const void* v, const ra_shape& s
     return launch_typed<T, OutT, 64, 128>(q, k, v, s, P, qo, ko, causal, scale, out, lse, st);
   if (s.d_qk == 128 && s.d_v == 64)
     return launch_typed<T, OutT, 128, 64>(q, k, v, s, P, qo, ko, causal, scale, out, lse, st);
-  if (s.d_qk == 192 && s.d_v == 128)
-    return launch_typed<T, OutT, 192, 128>(q, k, v, s, P, qo, ko, causal, scale, out, lse, st);
   return RA_ERR_UNSUPPORTED;
 }
 
@@ -183,14 +181,10 @@ int launch_simt_attention(const void* q, const void* k, const void* v, const ra_
                           int q_offset, int k_offset, int causal, float scale, void* out,
                           bool out_f32, float* lse, const DeviceInfo& dev, cudaStream_t stream) {
   (void)dev;
-  if (s.dtype == RA_F32)
-    return dispatch_dims<float, float>(q, k, v, s, P, q_offset, k_offset, causal, scale, out, lse,
-                                       stream);
-  if (out_f32)
-    return dispatch_dims<__nv_bfloat16, float>(q, k, v, s, P, q_offset, k_offset, causal, scale,
-                                               out, lse, stream);
-  return dispatch_dims<__nv_bfloat16, __nv_bfloat16>(q, k, v, s, P, q_offset, k_offset, causal,
-                                                     scale, out, lse, stream);
+  (void)out_f32;  // fp32 inputs give fp32 outputs
+  if (s.dtype != RA_F32) return RA_ERR_UNSUPPORTED;  // bf16 runs on the tensor-core kernel
+  return dispatch_dims<float, float>(q, k, v, s, P, q_offset, k_offset, causal, scale, out, lse,
+                                     stream);
 }
 
 }  // namespace ra

@@ -21,7 +21,7 @@
 // Warp w runs on sub-partition w % 4, so each sub-partition holds one warp of
 // each warpgroup.  The kernel is launched with 168 registers per thread;
 // setmaxnreg then moves registers from the third warpgroup to the two softmax
-// warpgroups within that launch allocation: 2 x 208 + 88 = 504 = 3 x 168 per
+// warpgroups within that launch allocation: 2 x 192 + 120 = 504 = 3 x 168 per
 // lane.  (setmaxnreg.inc waits until registers are free, so a split above the
 // launch allocation would never proceed; the launcher checks the compiled
 // register count against the split before every launch.)
@@ -56,8 +56,8 @@ constexpr int kBN = 128;          // keys per KV tile
 constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16 = 16 KB
 constexpr int kThreads = 384;
 constexpr int kRegsLaunch = 168;    // per thread at launch (384 threads, 1 CTA / SM)
-constexpr int kRegsSoftmax = 208;   // per thread, softmax warpgroups
-constexpr int kRegsOther = 88;      // per thread, producer / MMA warpgroup
+constexpr int kRegsSoftmax = 192;   // per thread, softmax warpgroups
+constexpr int kRegsOther = 120;     // per thread, producer / MMA warpgroup
 static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kRegsLaunch,
               "register split must fit the launch allocation");
 constexpr int kSmemLimit = 232448;

@@ -1,0 +1,69 @@
+"""Small, fixed launches of each kernel for profiler captures.
+
+    python -m ring_context_parallelism_ra_b200.profile_cases CASE [--reps N]
+
+Each case runs two warm-up launches and then N (default 1) launches of one
+kernel at a shape the bench uses, holding at most a few GB on the device:
+
+  prefill_cfg2   fused ring forward, causal MHA, 8 heads, n = 8192, d = 128,
+                 P = 4 (the bench's default workload, one launch per step)
+  prefill_gqa32k fused ring forward, causal GQA 32/8 heads, n = 32768, P = 8
+  decode_shard   pass-Q decode partial on one 131072-token shard of the
+                 1M-token cache (B = 4, 64/8 heads): one chunk-kernel launch
+                 and one merge launch, as one shard of the bench's decode step
+  merge_p8       LSE merge of 8 fp32 partials of shape [1, 32, 16384, 128]
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import ra
+from .workloads import make_qkv, make_workload_inputs, workload
+
+
+def _prefill(q, k, v, P, reps):
+    out = torch.empty((*q.shape[:3], v.shape[-1]), device=q.device, dtype=q.dtype)
+    lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
+    for _ in range(2 + reps):
+        ra.ring_forward(q, k, v, P, True, None, out, lse)
+    torch.cuda.synchronize()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["prefill_cfg2", "prefill_gqa32k", "decode_shard", "merge_p8"])
+    ap.add_argument("--reps", type=int, default=1)
+    args = ap.parse_args()
+    dev = "cuda"
+    if args.case == "prefill_cfg2":
+        wl = workload(2)
+        q, k, v = make_workload_inputs(wl, device=dev)
+        _prefill(q, k, v, wl.P, args.reps)
+    elif args.case == "prefill_gqa32k":
+        q, k, v = make_qkv(1, 32, 8, 32768, 32768, 128, 128, torch.bfloat16, seed=3, device=dev)
+        _prefill(q, k, v, 8, args.reps)
+    elif args.case == "decode_shard":
+        q, k, v = make_qkv(4, 64, 8, 1, 131072, 128, 128, torch.bfloat16, seed=4, device=dev)
+        ws = torch.empty(ra.decode_workspace_bytes(4, 64, 8, 131072), dtype=torch.uint8, device=dev)
+        o = torch.empty((4, 64, 128), device=dev)
+        l = torch.empty((4, 64), device=dev)
+        for _ in range(2 + args.reps):
+            ra.decode_partial(q, k, v, 0, 131072, None, ws, o, l)
+        torch.cuda.synchronize()
+    else:
+        g = torch.Generator(device=dev).manual_seed(5)
+        o = torch.randn((8, 1, 32, 16384, 128), device=dev, generator=g)
+        l = torch.randn((8, 1, 32, 16384), device=dev, generator=g)
+        out = torch.empty((1, 32, 16384, 128), device=dev, dtype=torch.bfloat16)
+        lse = torch.empty((1, 32, 16384), device=dev)
+        for _ in range(2 + args.reps):
+            ra.lse_merge(o, l, torch.bfloat16, out, lse)
+        torch.cuda.synchronize()
+    assert ra.get_status() == ra.RA_OK
+    print(f"{args.case}: ok")
+
+
+if __name__ == "__main__":
+    main()
