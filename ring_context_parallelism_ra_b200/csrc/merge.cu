@@ -76,20 +76,110 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
   }
 }
 
+// Few rows, many partials (the chunk partials of one decode shard): the
+// row-per-warp kernel above would leave the GPU nearly idle and walk P
+// partials serially.  Here eight warps share each row group, warp w taking
+// partials p = w, w + 8, ...; each warp merges its subset relative to its own
+// max, and the eight sub-results are merged the same way through shared memory
+// (the merge is associative).
+template <typename OutT>
+__global__ void __launch_bounds__(256) lse_merge_splitp_kernel(const float* __restrict__ o_parts,
+                                                               const float* __restrict__ lse_parts,
+                                                               int P, long long rows, int d_v,
+                                                               OutT* __restrict__ out,
+                                                               float* __restrict__ lse_out) {
+  constexpr int kWarps = 8;
+  __shared__ float4 s_acc[kWarps][32];
+  __shared__ float s_m[kWarps][32];
+  __shared__ float s_w[kWarps][32];
+  const int lanes_per_row = d_v >> 2;
+  const int rows_per_warp = 32 / lanes_per_row;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / lanes_per_row;
+  const int col = (lane % lanes_per_row) * 4;
+  const long long part_stride = rows * d_v;
+  for (long long r0 = static_cast<long long>(blockIdx.x) * rows_per_warp; r0 < rows;
+       r0 += static_cast<long long>(gridDim.x) * rows_per_warp) {
+    const long long r = r0 + sub;
+    float m = -INFINITY, w_sum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < rows) {
+      for (int p = warp; p < P; p += kWarps) m = fmaxf(m, __ldg(lse_parts + p * rows + r));
+      if (m != -INFINITY) {
+        const float* src = o_parts + r * d_v + col;
+#pragma unroll 4
+        for (int p = warp; p < P; p += kWarps) {
+          const float l = __ldg(lse_parts + p * rows + r);
+          const float4 o = __ldcs(reinterpret_cast<const float4*>(src + p * part_stride));
+          const float w = (l == -INFINITY) ? 0.f : expf(l - m);
+          w_sum += w;
+          acc.x = fmaf(w, o.x, acc.x);
+          acc.y = fmaf(w, o.y, acc.y);
+          acc.z = fmaf(w, o.z, acc.z);
+          acc.w = fmaf(w, o.w, acc.w);
+        }
+      }
+    }
+    s_acc[warp][lane] = acc;
+    s_m[warp][lane] = m;
+    s_w[warp][lane] = w_sum;
+    __syncthreads();
+    if (warp == 0 && r < rows) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, s_m[w][lane]);
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      float tot = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          const float mw = s_m[w][lane];
+          const float f = (mw == -INFINITY) ? 0.f : expf(mw - M);
+          const float4 a = s_acc[w][lane];
+          tot = fmaf(f, s_w[w][lane], tot);
+          o.x = fmaf(f, a.x, o.x);
+          o.y = fmaf(f, a.y, o.y);
+          o.z = fmaf(f, a.z, o.z);
+          o.w = fmaf(f, a.w, o.w);
+        }
+        const float inv = 1.f / tot;
+        o.x *= inv; o.y *= inv; o.z *= inv; o.w *= inv;
+      }
+      store4<OutT>(out + r * d_v + col, o);
+      if (lse_out != nullptr && col == 0) lse_out[r] = (M == -INFINITY) ? -INFINITY : M + logf(tot);
+    }
+    __syncthreads();
+  }
+}
+
 int launch_lse_merge(const float* o_parts, const float* lse_parts, int P, long long rows, int d_v,
                      void* out, ra_dtype out_dtype, float* lse, int num_sms, cudaStream_t stream) {
   const int threads = 256;
-  const int rows_per_cta = (threads / 32) * (32 / (d_v / 4));
-  long long want = (rows + rows_per_cta - 1) / rows_per_cta;
-  long long cap = static_cast<long long>(num_sms) * 8;   // 8 resident CTAs / SM
-  int grid = static_cast<int>(want < cap ? want : cap);
-  if (grid < 1) grid = 1;
-  if (out_dtype == RA_F32) {
-    lse_merge_kernel<float><<<grid, threads, 0, stream>>>(o_parts, lse_parts, P, rows, d_v,
-                                                          static_cast<float*>(out), lse);
+  const int rows_per_warp = 32 / (d_v / 4);
+  const long long warps_needed = (rows + rows_per_warp - 1) / rows_per_warp;
+  if (P >= 8 && warps_needed < static_cast<long long>(num_sms) * 16) {
+    // few rows: eight warps per row group, each over a subset of the partials
+    const int grid = static_cast<int>(warps_needed);
+    if (out_dtype == RA_F32)
+      lse_merge_splitp_kernel<float><<<grid, threads, 0, stream>>>(
+          o_parts, lse_parts, P, rows, d_v, static_cast<float*>(out), lse);
+    else
+      lse_merge_splitp_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
+          o_parts, lse_parts, P, rows, d_v, static_cast<__nv_bfloat16*>(out), lse);
   } else {
-    lse_merge_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
-        o_parts, lse_parts, P, rows, d_v, static_cast<__nv_bfloat16*>(out), lse);
+    const int rows_per_cta = (threads / 32) * rows_per_warp;
+    long long want = (rows + rows_per_cta - 1) / rows_per_cta;
+    long long cap = static_cast<long long>(num_sms) * 8;   // 8 resident CTAs / SM
+    int grid = static_cast<int>(want < cap ? want : cap);
+    if (grid < 1) grid = 1;
+    if (out_dtype == RA_F32) {
+      lse_merge_kernel<float><<<grid, threads, 0, stream>>>(o_parts, lse_parts, P, rows, d_v,
+                                                            static_cast<float*>(out), lse);
+    } else {
+      lse_merge_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
+          o_parts, lse_parts, P, rows, d_v, static_cast<__nv_bfloat16*>(out), lse);
+    }
   }
   note_launch();
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;

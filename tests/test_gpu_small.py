@@ -52,6 +52,23 @@ def test_lse_merge_matches_oracle(P, dv, out_dtype):
     assert (out[1, 2, 7] == 0).all() and lse[1, 2, 7].item() == -math.inf
 
 
+@pytest.mark.parametrize("P,B,H,n,dv", [(8, 1, 8, 4096, 128),    # many rows: one warp per row
+                                        (12, 1, 3, 37, 64),      # few rows, odd count: split-P
+                                        (64, 4, 64, 1, 128),     # decode chunk partials
+                                        (9, 2, 2, 5, 32)])
+def test_lse_merge_both_kernels(P, B, H, n, dv):
+    g = torch.Generator().manual_seed(P * 1000 + n)
+    o = torch.randn((P, B, H, n, dv), generator=g)
+    l = torch.randn((P, B, H, n), generator=g) * 4
+    l[P - 1, 0, 0, 0] = -math.inf
+    l[:, B - 1, H - 1, n - 1] = -math.inf
+    for out_dtype in (torch.float32, torch.bfloat16):
+        out, lse = ra.lse_merge(o.to(DEV), l.to(DEV), out_dtype)
+        want_o, want_l = oracle_merge(o.numpy(), l.numpy())
+        check_out(out, want_o, "f32" if out_dtype == torch.float32 else "bf16")
+        check_lse(lse, want_l)
+
+
 def test_decode_merge_matches_oracle():
     g = torch.Generator().manual_seed(7)
     P, B, H, d = 8, 4, 64, 128
