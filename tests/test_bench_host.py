@@ -1,0 +1,97 @@
+"""CPU tests of bench.py's host logic: the multi-rank (replica) helpers over
+gloo with world size 2, the per-rank input seeds, and the reference arm's
+output contract."""
+import dataclasses
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from ring_context_parallelism_ra_b200.workloads import make_workload_inputs, workload  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        got = bench.max_over_ranks(1.5 + rank, world)
+        out_q.put((rank, got))
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=5) for _ in range(2))
+    assert res == {0: 2.5, 1: 2.5}
+
+
+def test_replica_seeds_give_different_inputs():
+    wl = workload(1)
+    q0, _, _ = make_workload_inputs(wl)
+    q1, _, _ = make_workload_inputs(dataclasses.replace(wl, seed=wl.seed + 1000))
+    q0b, _, _ = make_workload_inputs(wl)
+    assert torch.equal(q0, q0b)
+    assert not torch.equal(q0, q1)
+
+
+def test_reference_arm_other_ranks_print_nothing():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], cwd=ROOT, env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
+
+
+def test_reference_arm_line():
+    env = dict(os.environ, RA_ORACLE_BUDGET_S="0.6")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2",
+                        "--warmup", "3"], cwd=ROOT, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "config", "cpu_baseline", "e2e"):
+        assert key in line
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
+    assert line["config"]["workload"] == workload(2).name
+
+
+def test_flop_and_byte_counts_match_oracle_formulas():
+    from oracle.costs import kv_cache_bytes, prefill_flops as oracle_flops
+    from ring_context_parallelism_ra_b200.workloads import decode_kv_bytes, prefill_flops
+    for key in (1, 2, 3, 5):
+        wl = workload(key)
+        assert prefill_flops(wl) == oracle_flops(wl.B, wl.n, wl.d_qk, wl.d_v, wl.Hq, wl.causal)
+    wl = workload(4)
+    assert decode_kv_bytes(wl) == wl.B * kv_cache_bytes(1, wl.Hkv, wl.d_qk, wl.n, 2)
+    assert decode_kv_bytes(wl) == 17179869184
