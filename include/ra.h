@@ -90,6 +90,22 @@ int ra_block_partial(const void* q, const void* k, const void* v, const ra_shape
                      float* o_part, float* lse_part, void* stream);
 
 /*
+ * ra_block_partial_strided -- ra_block_partial with positions spaced by
+ * pos_stride: query row t is token q_offset + t * pos_stride and key u is
+ * token k_offset + u * pos_stride.  With the striped split of page
+ * "LLM长文本推理Ring Attention环形注意力机制实现与优化", section on tuning
+ * (Striped Attention interleaves token positions across devices), partition
+ * i holds tokens i, i + P, i + 2P, ...: its block against partition j is this
+ * call with q_offset = i, k_offset = j, pos_stride = P.  Every such block is
+ * about half visible, which balances causal work across the P devices.
+ *   pos_stride  : >= 1 (1 gives ra_block_partial).
+ *   Other arguments, outputs and errors as ra_block_partial.
+ */
+int ra_block_partial_strided(const void* q, const void* k, const void* v, const ra_shape* shape,
+                             int q_offset, int k_offset, int pos_stride, int causal, float scale,
+                             float* o_part, float* lse_part, void* stream);
+
+/*
  * ra_lse_merge -- N-way merge of normalised partials over disjoint key sets
  * (step a6), the closed form of the beta / gamma update of page
  * "LLM长文本推理Ring Attention环形注意力机制实现与优化", section
@@ -120,6 +136,20 @@ int ra_lse_merge(const float* o_parts, const float* lse_parts, int P, const ra_s
  */
 int ra_ring_forward(const void* q, const void* k, const void* v, int P, int causal, float scale,
                     void* out, float* lse, const ra_shape* shape, void* stream);
+
+/*
+ * ra_ring_forward_striped -- the fused ring over a striped split (same page
+ * and section as ra_block_partial_strided): the tensors hold the P
+ * partitions one after another, partition i being tokens i, i + P, i + 2P,
+ * ... in order, so tensor row R = i * (n / P) + r is token r * P + i.  Output
+ * rows are in the same order.  The causal mask follows the token positions;
+ * no partition block is skipped whole (each is half visible), tiles are.
+ *   Arguments as ra_ring_forward; additionally (n / P) % 256 == 0, else
+ *   RA_ERR_UNSUPPORTED.
+ */
+int ra_ring_forward_striped(const void* q, const void* k, const void* v, int P, int causal,
+                            float scale, void* out, float* lse, const ra_shape* shape,
+                            void* stream);
 
 /*
  * ra_decode_workspace_bytes -- bytes of device workspace ra_decode_partial

@@ -74,13 +74,17 @@ def _rows_attention(q_rows, k, v, scale, causal, q_pos, k_pos):
 
 
 def attention(q, k, v, scale: float, causal: bool, q_offset: int = 0,
-              k_offset: int = 0, rows=None, heads=None, row_chunk: int = 512):
+              k_offset: int = 0, rows=None, heads=None, row_chunk: int = 512,
+              q_positions=None, k_positions=None):
     """fp64 attention over BHSD tensors.
 
     q [B, H_q, n_q, dqk], k [B, H_kv, n_k, dqk], v [B, H_kv, n_k, dv] (numpy
     or torch, any float dtype; converted exactly to fp64 per head).
     ``rows``: optional 1-D array of query row indices (default: all rows).
     ``heads``: optional list of query heads (default: all).
+    ``q_positions`` / ``k_positions``: optional absolute token positions of
+    every query row / key (default q_offset + t, k_offset + u); the causal
+    rule compares these.
     Returns (O [B, len(heads), len(rows), dv], LSE [B, len(heads), len(rows)]).
     """
     B, h_q, n_q, dqk = q.shape
@@ -93,7 +97,10 @@ def attention(q, k, v, scale: float, causal: bool, q_offset: int = 0,
     heads = list(range(h_q)) if heads is None else list(heads)
     out = np.zeros((B, len(heads), len(rows), dv))
     lse = np.zeros((B, len(heads), len(rows)))
-    k_pos = k_offset + np.arange(n_k, dtype=np.int64)
+    k_pos = (k_offset + np.arange(n_k, dtype=np.int64) if k_positions is None
+             else np.asarray(k_positions, dtype=np.int64))
+    q_pos_all = (q_offset + np.arange(n_q, dtype=np.int64) if q_positions is None
+                 else np.asarray(q_positions, dtype=np.int64))
     for b in range(B):
         cached_g, kk, vv = None, None, None
         for hi, h in enumerate(heads):
@@ -105,7 +112,7 @@ def attention(q, k, v, scale: float, causal: bool, q_offset: int = 0,
                 r = rows[c0:c0 + row_chunk]
                 q_rows = _as_f64(qh[r])
                 o_c, l_c = _rows_attention(q_rows, kk, vv, scale, causal,
-                                           q_offset + r, k_pos)
+                                           q_pos_all[r], k_pos)
                 out[b, hi, c0:c0 + len(r)] = o_c
                 lse[b, hi, c0:c0 + len(r)] = l_c
     return out, lse

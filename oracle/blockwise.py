@@ -34,8 +34,8 @@ import numpy as np
 
 from .attention import _as_f64, gqa_group
 
-__all__ = ["partition_bounds", "ring_order", "block_scores",
-           "ring_attention_normalised", "ring_attention_online"]
+__all__ = ["partition_bounds", "ring_order", "block_scores", "striped_positions",
+           "ring_attention_normalised", "ring_attention_online", "striped_block_visible"]
 
 
 def partition_bounds(n: int, P: int):
@@ -49,6 +49,22 @@ def partition_bounds(n: int, P: int):
 def ring_order(P: int, i: int):
     """KV partitions met by query partition i, in step order s = 0..P-1."""
     return [(i - s) % P for s in range(P)]
+
+
+def striped_positions(n: int, P: int, i: int):
+    """Token positions held by partition i of a striped split (page
+    "LLM长文本推理…", tuning section: Striped Attention hands sequence positions
+    to the devices interleaved): i, i + P, i + 2P, ..."""
+    if P <= 0 or n % P != 0:
+        raise ValueError(f"n={n} is not divisible into P={P} equal partitions")
+    return np.arange(i, n, P, dtype=np.int64)
+
+
+def striped_block_visible(n: int, P: int, i: int, j: int) -> int:
+    """Number of visible (query, key) pairs in block (Q_i, KV_j) of a striped
+    split, counted from the explicit positions."""
+    qp, kp = striped_positions(n, P, i), striped_positions(n, P, j)
+    return int((kp[None, :] <= qp[:, None]).sum())
 
 
 def block_scores(q_blk, k_blk, scale, causal, q_pos, k_pos):

@@ -24,19 +24,37 @@ namespace ra {
 
 enum : int8_t { kSkip = 0, kPartial = 1, kFull = 2 };
 
+// Floor division (rounds toward -inf, also for a negative numerator).
+RA_HD long long floor_div(long long a, long long b) {
+  const long long q = a / b;
+  return (q * b != a && ((a < 0) != (b < 0))) ? q - 1 : q;
+}
+
 // q0, q_len: first row and row count of the tile (rows beyond n_q excluded
-// by the caller); k0, k_len likewise for keys.  Offsets are absolute token
-// positions of row 0 / key 0.
+// by the caller); k0, k_len likewise for keys.  Row t of the tensor sits at
+// absolute position q_offset + t * stride, key u at k_offset + u * stride
+// (stride 1: contiguous tokens; stride P: a partition of a striped split,
+// where token p of the sequence goes to partition p mod P).  Positions grow
+// with the index, so the corner pairs still decide the class.
 RA_HD int8_t tile_class(long long q0, long long q_len, long long k0, long long k_len,
-                        long long q_offset, long long k_offset, int causal) {
+                        long long q_offset, long long k_offset, int causal,
+                        long long stride = 1) {
   if (!causal) return kFull;
-  const long long first_q = q_offset + q0;
-  const long long last_q = first_q + q_len - 1;
-  const long long first_k = k_offset + k0;
-  const long long last_k = first_k + k_len - 1;
+  const long long first_q = q_offset + q0 * stride;
+  const long long last_q = first_q + (q_len - 1) * stride;
+  const long long first_k = k_offset + k0 * stride;
+  const long long last_k = first_k + (k_len - 1) * stride;
   if (first_k > last_q) return kSkip;
   if (last_k <= first_q) return kFull;
   return kPartial;
+}
+
+// Number of leading keys of a tile (key indices k0, k0 + 1, ...) visible to
+// query row t: key u is visible iff k_offset + u * stride <= q_offset + t *
+// stride, i.e. u - t <= floor((q_offset - k_offset) / stride).  Not clipped.
+RA_HD long long visible_keys(long long t, long long k0, long long q_offset, long long k_offset,
+                             long long stride) {
+  return floor_div(q_offset - k_offset, stride) + t - k0 + 1;
 }
 
 }  // namespace ra

@@ -25,16 +25,21 @@ int device_info(DeviceInfo* out);
 int launch_lse_merge(const float* o_parts, const float* lse_parts, int P, long long rows, int d_v,
                      void* out, ra_dtype out_dtype, float* lse, int num_sms, cudaStream_t stream);
 
-// Exact-fp32 (SIMT) attention: block partial (P = 1, offsets) or the fused
-// ring (P >= 1, offsets 0).  out_f32 selects fp32 output (partials).
+// Attention launchers.  Positions: query row t is token q_offset + t * stride
+// and key u is token k_offset + u * stride (block partial: P = 1); with
+// striped = 1 (fused ring) row r of partition i is token r * P + i and the
+// offsets / stride arguments are ignored.  out_f32 selects fp32 output.
+// Exact-fp32 (SIMT) attention for fp32 inputs:
 int launch_simt_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
-                          int q_offset, int k_offset, int causal, float scale, void* out,
-                          bool out_f32, float* lse, const DeviceInfo& dev, cudaStream_t stream);
+                          int q_offset, int k_offset, long long stride, int causal, int striped,
+                          float scale, void* out, bool out_f32, float* lse,
+                          const DeviceInfo& dev, cudaStream_t stream);
 
 // Tensor-core (tcgen05) attention, bf16 inputs.
 int launch_tc_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
-                        int q_offset, int k_offset, int causal, float scale, void* out,
-                        bool out_f32, float* lse, const DeviceInfo& dev, cudaStream_t stream);
+                        int q_offset, int k_offset, long long stride, int causal, int striped,
+                        float scale, void* out, bool out_f32, float* lse, const DeviceInfo& dev,
+                        cudaStream_t stream);
 
 // Decode: chunk partials of one shard into the workspace, then the merge.
 size_t decode_workspace_bytes(const ra_shape& s);

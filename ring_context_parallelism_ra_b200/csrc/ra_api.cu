@@ -48,16 +48,41 @@ int check_attention_dims(const ra_shape* s) {
 }
 
 int dispatch_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
-                       int q_offset, int k_offset, int causal, float scale, void* out,
-                       bool out_f32, float* lse, cudaStream_t st) {
+                       int q_offset, int k_offset, long long stride, int causal, int striped,
+                       float scale, void* out, bool out_f32, float* lse, cudaStream_t st) {
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc != RA_OK) return rc;
   if (s.dtype == RA_BF16)
-    return launch_tc_attention(q, k, v, s, P, q_offset, k_offset, causal, scale, out, out_f32,
-                               lse, dev, st);
-  return launch_simt_attention(q, k, v, s, P, q_offset, k_offset, causal, scale, out, out_f32,
-                               lse, dev, st);
+    return launch_tc_attention(q, k, v, s, P, q_offset, k_offset, stride, causal, striped, scale,
+                               out, out_f32, lse, dev, st);
+  return launch_simt_attention(q, k, v, s, P, q_offset, k_offset, stride, causal, striped, scale,
+                               out, out_f32, lse, dev, st);
+}
+
+int check_block_args(const void* q, const void* k, const void* v, const ra_shape* shape,
+                     int q_offset, int k_offset, int causal, const float* o_part,
+                     const float* lse_part) {
+  int rc = check_common(shape);
+  if (rc != RA_OK) return rc;
+  if (!q || !k || !v || !o_part || !lse_part) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
+    return RA_ERR_INVALID;
+  if ((causal != 0 && causal != 1) || q_offset < 0 || k_offset < 0) return RA_ERR_INVALID;
+  return check_attention_dims(shape);
+}
+
+int check_ring_args(const void* q, const void* k, const void* v, int P, int causal,
+                    const void* out, const float* lse, const ra_shape* shape) {
+  int rc = check_common(shape);
+  if (rc != RA_OK) return rc;
+  if (!q || !k || !v || !out) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return RA_ERR_INVALID;
+  if (P < 1 || shape->n_q != shape->n_k || shape->n_q % P != 0) return RA_ERR_INVALID;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID;
+  return check_attention_dims(shape);
 }
 
 __global__ void block_class_kernel(int n_q, int n_k, int q_block, int k_block, int q_offset,
@@ -143,32 +168,38 @@ extern "C" {
 int ra_block_partial(const void* q, const void* k, const void* v, const ra_shape* shape,
                      int q_offset, int k_offset, int causal, float scale, float* o_part,
                      float* lse_part, void* stream) {
-  int rc = check_common(shape);
+  const int rc = check_block_args(q, k, v, shape, q_offset, k_offset, causal, o_part, lse_part);
   if (rc != RA_OK) return rc;
-  if (!q || !k || !v || !o_part || !lse_part) return RA_ERR_INVALID;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
-    return RA_ERR_INVALID;
-  if ((causal != 0 && causal != 1) || q_offset < 0 || k_offset < 0) return RA_ERR_INVALID;
-  rc = check_attention_dims(shape);
+  return dispatch_attention(q, k, v, *shape, 1, q_offset, k_offset, 1, causal, 0, scale, o_part,
+                            true, lse_part, static_cast<cudaStream_t>(stream));
+}
+
+int ra_block_partial_strided(const void* q, const void* k, const void* v, const ra_shape* shape,
+                             int q_offset, int k_offset, int pos_stride, int causal, float scale,
+                             float* o_part, float* lse_part, void* stream) {
+  const int rc = check_block_args(q, k, v, shape, q_offset, k_offset, causal, o_part, lse_part);
   if (rc != RA_OK) return rc;
-  return dispatch_attention(q, k, v, *shape, 1, q_offset, k_offset, causal, scale, o_part, true,
-                            lse_part, static_cast<cudaStream_t>(stream));
+  if (pos_stride < 1) return RA_ERR_INVALID;
+  return dispatch_attention(q, k, v, *shape, 1, q_offset, k_offset, pos_stride, causal, 0, scale,
+                            o_part, true, lse_part, static_cast<cudaStream_t>(stream));
 }
 
 int ra_ring_forward(const void* q, const void* k, const void* v, int P, int causal, float scale,
                     void* out, float* lse, const ra_shape* shape, void* stream) {
-  int rc = check_common(shape);
+  const int rc = check_ring_args(q, k, v, P, causal, out, lse, shape);
   if (rc != RA_OK) return rc;
-  if (!q || !k || !v || !out) return RA_ERR_INVALID;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (lse && !aligned16(lse)))
-    return RA_ERR_INVALID;
-  if (P < 1 || shape->n_q != shape->n_k || shape->n_q % P != 0) return RA_ERR_INVALID;
-  if (causal != 0 && causal != 1) return RA_ERR_INVALID;
-  rc = check_attention_dims(shape);
+  return dispatch_attention(q, k, v, *shape, P, 0, 0, 1, causal, 0, scale, out,
+                            shape->dtype == RA_F32, lse, static_cast<cudaStream_t>(stream));
+}
+
+int ra_ring_forward_striped(const void* q, const void* k, const void* v, int P, int causal,
+                            float scale, void* out, float* lse, const ra_shape* shape,
+                            void* stream) {
+  const int rc = check_ring_args(q, k, v, P, causal, out, lse, shape);
   if (rc != RA_OK) return rc;
-  return dispatch_attention(q, k, v, *shape, P, 0, 0, causal, scale, out, shape->dtype == RA_F32,
-                            lse, static_cast<cudaStream_t>(stream));
+  if ((shape->n_q / P) % 256 != 0) return RA_ERR_UNSUPPORTED;
+  return dispatch_attention(q, k, v, *shape, P, 0, 0, P, causal, 1, scale, out,
+                            shape->dtype == RA_F32, lse, static_cast<cudaStream_t>(stream));
 }
 
 int ra_lse_merge(const float* o_parts, const float* lse_parts, int P, const ra_shape* shape,

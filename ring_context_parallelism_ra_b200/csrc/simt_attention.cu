@@ -31,8 +31,8 @@ constexpr size_t simt_smem_bytes() {
 template <typename T, typename OutT, int DQK, int DV>
 __global__ void __launch_bounds__(kThreads) simt_attention_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, int Hq, int Hkv,
-    int n_q, int n_k, int P, int q_offset, int k_offset, int causal, float scale_log2,
-    OutT* __restrict__ out, float* __restrict__ lse) {
+    int n_q, int n_k, int P, int q_offset, int k_offset, long long stride, int causal,
+    int striped, float scale_log2, OutT* __restrict__ out, float* __restrict__ lse) {
   constexpr int QS = DQK + 1;
   constexpr int PS = kBN + 1;
   constexpr int CPT = DV / 4;  // output columns per thread
@@ -61,7 +61,6 @@ __global__ void __launch_bounds__(kThreads) simt_attention_kernel(
     Qs[rr * QS + cc] = (rr < rows_here) ? to_f32(qh[static_cast<long long>(row0 + rr) * DQK + cc]) : 0.f;
   }
 
-  const long long q_pos = static_cast<long long>(q_offset) + row0 + r;
   float m = -INFINITY, l = 0.f;
   float o[CPT];
 #pragma unroll
@@ -70,14 +69,21 @@ __global__ void __launch_bounds__(kThreads) simt_attention_kernel(
   const int part_q = n_q / P;
   const int part_k = n_k / P;
   const int i = min(row0 / part_q, P - 1);
+  // positions: row t is token qoff + t * st, key u is token koff + u * st;
+  // in the striped split row R of partition p is token R * P + p * (1 - L * P)
+  const long long st = striped ? P : stride;
+  const long long qoff = striped ? static_cast<long long>(i) * (1 - static_cast<long long>(part_q) * P)
+                                 : static_cast<long long>(q_offset);
 
   for (int s = 0; s < P; ++s) {
     const int j = (i - s + P) % P;
     const int kbeg = j * part_k;
     const int kend = kbeg + part_k;
+    const long long koff = striped ? static_cast<long long>(j) * (1 - static_cast<long long>(part_k) * P)
+                                   : static_cast<long long>(k_offset);
     for (int kt = kbeg; kt < kend; kt += kBN) {
       const int klen = min(kBN, kend - kt);
-      const int8_t cls = tile_class(row0, rows_here, kt, klen, q_offset, k_offset, causal);
+      const int8_t cls = tile_class(row0, rows_here, kt, klen, qoff, koff, causal, st);
       if (cls == kSkip) continue;
       __syncthreads();  // previous tile fully consumed (and Q stored, first time)
       for (int e = tid; e < kBN * DQK; e += kThreads) {
@@ -90,6 +96,7 @@ __global__ void __launch_bounds__(kThreads) simt_attention_kernel(
       }
       __syncthreads();
 
+      const long long lim = (cls == kFull) ? klen : visible_keys(row0 + r, kt, qoff, koff, st);
       float sc[kBN / 4];
       float mx = -INFINITY;
 #pragma unroll
@@ -101,8 +108,7 @@ __global__ void __launch_bounds__(kThreads) simt_attention_kernel(
 #pragma unroll 8
         for (int kk = 0; kk < DQK; ++kk) acc = fmaf(qr[kk], kr[kk], acc);
         float sv = acc * scale_log2;
-        const bool vis = jl < klen &&
-                         (cls == kFull || static_cast<long long>(k_offset) + kt + jl <= q_pos);
+        const bool vis = jl < klen && jl < lim;
         sv = vis ? sv : -INFINITY;
         sc[mm] = sv;
         mx = fmaxf(mx, sv);
@@ -146,7 +152,8 @@ __global__ void __launch_bounds__(kThreads) simt_attention_kernel(
 
 template <typename T, typename OutT, int DQK, int DV>
 int launch_typed(const void* q, const void* k, const void* v, const ra_shape& s, int P, int q_offset,
-                 int k_offset, int causal, float scale, void* out, float* lse, cudaStream_t stream) {
+                 int k_offset, long long stride, int causal, int striped, float scale, void* out,
+                 float* lse, cudaStream_t stream) {
   auto kern = simt_attention_kernel<T, OutT, DQK, DV>;
   const size_t smem = simt_smem_bytes<DQK, DV>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -155,36 +162,42 @@ int launch_typed(const void* q, const void* k, const void* v, const ra_shape& s,
   dim3 grid((s.n_q + kBM - 1) / kBM, s.B * s.Hq);
   kern<<<grid, kThreads, smem, stream>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                                          static_cast<const T*>(v), s.Hq, s.Hkv, s.n_q, s.n_k, P,
-                                         q_offset, k_offset, causal, scale * kLog2e,
-                                         static_cast<OutT*>(out), lse);
+                                         q_offset, k_offset, stride, causal, striped,
+                                         scale * kLog2e, static_cast<OutT*>(out), lse);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 template <typename T, typename OutT>
 int dispatch_dims(const void* q, const void* k, const void* v, const ra_shape& s, int P, int qo,
-                  int ko, int causal, float scale, void* out, float* lse, cudaStream_t st) {
+                  int ko, long long st, int causal, int striped, float scale, void* out, float* lse,
+                  cudaStream_t stm) {
   if (s.d_qk == 64 && s.d_v == 64)
-    return launch_typed<T, OutT, 64, 64>(q, k, v, s, P, qo, ko, causal, scale, out, lse, st);
+    return launch_typed<T, OutT, 64, 64>(q, k, v, s, P, qo, ko, st, causal, striped, scale, out,
+                                         lse, stm);
   if (s.d_qk == 128 && s.d_v == 128)
-    return launch_typed<T, OutT, 128, 128>(q, k, v, s, P, qo, ko, causal, scale, out, lse, st);
+    return launch_typed<T, OutT, 128, 128>(q, k, v, s, P, qo, ko, st, causal, striped, scale, out,
+                                           lse, stm);
   if (s.d_qk == 64 && s.d_v == 128)
-    return launch_typed<T, OutT, 64, 128>(q, k, v, s, P, qo, ko, causal, scale, out, lse, st);
+    return launch_typed<T, OutT, 64, 128>(q, k, v, s, P, qo, ko, st, causal, striped, scale, out,
+                                          lse, stm);
   if (s.d_qk == 128 && s.d_v == 64)
-    return launch_typed<T, OutT, 128, 64>(q, k, v, s, P, qo, ko, causal, scale, out, lse, st);
+    return launch_typed<T, OutT, 128, 64>(q, k, v, s, P, qo, ko, st, causal, striped, scale, out,
+                                          lse, stm);
   return RA_ERR_UNSUPPORTED;
 }
 
 }  // namespace
 
 int launch_simt_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
-                          int q_offset, int k_offset, int causal, float scale, void* out,
-                          bool out_f32, float* lse, const DeviceInfo& dev, cudaStream_t stream) {
+                          int q_offset, int k_offset, long long stride, int causal, int striped,
+                          float scale, void* out, bool out_f32, float* lse,
+                          const DeviceInfo& dev, cudaStream_t stream) {
   (void)dev;
   (void)out_f32;  // fp32 inputs give fp32 outputs
   if (s.dtype != RA_F32) return RA_ERR_UNSUPPORTED;  // bf16 runs on the tensor-core kernel
-  return dispatch_dims<float, float>(q, k, v, s, P, q_offset, k_offset, causal, scale, out, lse,
-                                     stream);
+  return dispatch_dims<float, float>(q, k, v, s, P, q_offset, k_offset, stride, causal, striped,
+                                     scale, out, lse, stream);
 }
 
 }  // namespace ra

@@ -81,6 +81,8 @@ struct Cfg {
 struct TcArgs {
   int B, Hq, Hkv, n_q, n_k, P;
   int q_offset, k_offset, causal;
+  int striped;        // 1: row r of partition i is token r * P + i (needs n / P % 256 == 0)
+  long long stride;   // position stride (1 contiguous; P striped; any for a strided block)
   float scale_log2;
   void* out;          // [B*Hq, n_q, DV] bf16 or fp32
   float* lse;         // [B*Hq, n_q] or null
@@ -92,8 +94,19 @@ struct TcArgs {
 struct Item {
   int bh, b, g;
   int q0[2], qlen[2];
-  int i;  // ring partition of the item's first row
+  int i;           // ring partition of the item's first row
+  long long qoff;  // query position = qoff + row * stride
 };
+
+// Position offset of a partition: contiguous tokens use the call's offsets;
+// in the striped split (stride P), tensor row R of partition p (R - p * L its
+// index inside the partition) is token (R - p * L) * P + p = R * P + p * (1 -
+// L * P).
+__device__ __forceinline__ long long pos_stride(const TcArgs& a) { return a.stride; }
+__device__ __forceinline__ long long part_offset(const TcArgs& a, int p, int n, int base) {
+  return a.striped ? static_cast<long long>(p) * (1 - static_cast<long long>(n / a.P) * a.P)
+                   : static_cast<long long>(base);
+}
 
 __device__ __forceinline__ bool item_at(const TcArgs& a, int round, Item& it) {
   const int G = gridDim.x;
@@ -114,43 +127,51 @@ __device__ __forceinline__ bool item_at(const TcArgs& a, int round, Item& it) {
   const int Lq = a.n_q / a.P;
   const int i = it.q0[0] / Lq;
   it.i = i < a.P - 1 ? i : a.P - 1;
+  it.qoff = part_offset(a, it.i, a.n_q, a.q_offset);
   return true;
 }
 
 // The KV tiles an item visits, in ring order; every role runs this same walk.
 struct TileWalk {
-  int s, kt, kend;
+  int s, j, kt, kend;
+  long long koff;  // key position = koff + key index * stride, partition j
   __device__ __forceinline__ void start(const TcArgs& a, const Item& it) {
     const int Lk = a.n_k / a.P;
     s = 0;
-    kt = it.i * Lk;
+    j = it.i;
+    kt = j * Lk;
     kend = kt + Lk;
+    koff = part_offset(a, j, a.n_k, a.k_offset);
   }
-  // Next tile with at least one active query tile: kt0, klen, class per tile.
+  // Next tile with at least one active query tile: kt0, klen, the partition's
+  // key offset and the class per query tile.
   __device__ __forceinline__ bool next(const TcArgs& a, const Item& it, int& kt0, int& klen,
-                                       int8_t (&cls)[2]) {
+                                       long long& koff_out, int8_t (&cls)[2]) {
     const int Lk = a.n_k / a.P;
+    const long long st = pos_stride(a);
     while (true) {
       if (kt >= kend) {
         if (++s >= a.P) return false;
-        const int j = (it.i - s + a.P) % a.P;
+        j = (it.i - s + a.P) % a.P;
         kt = j * Lk;
         kend = kt + Lk;
+        koff = part_offset(a, j, a.n_k, a.k_offset);
         continue;
       }
       const int len = kend - kt < kBN ? kend - kt : kBN;
       for (int t = 0; t < 2; ++t)
-        cls[t] = it.qlen[t] > 0 ? tile_class(it.q0[t], it.qlen[t], kt, len, a.q_offset,
-                                              a.k_offset, a.causal)
+        cls[t] = it.qlen[t] > 0 ? tile_class(it.q0[t], it.qlen[t], kt, len, it.qoff, koff,
+                                              a.causal, st)
                                 : static_cast<int8_t>(kSkip);
       if (cls[0] == kSkip && cls[1] == kSkip) {
-        // keys only grow inside a partition: with a causal mask nothing
-        // later in this partition is visible either
+        // key positions only grow inside a partition: with a causal mask
+        // nothing later in this partition is visible either
         if (a.causal) kt = kend; else kt += kBN;
         continue;
       }
       kt0 = kt;
       klen = len;
+      koff_out = koff;
       kt += kBN;
       return true;
     }
@@ -256,9 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
         TileWalk w;
         w.start(a, it);
         int kt, klen;
+        long long koff;
         int8_t cls[2];
         bool ok = true;
-        while (ok && w.next(a, it, kt, klen, cls)) {
+        while (ok && w.next(a, it, kt, klen, koff, cls)) {
           for (int part = 0; part < 2 && ok; ++part) {  // K then V
             const int s = ld % NSLOT;
             if (!mbar_wait(&slot_empty[s], ((ld / NSLOT) & 1) ^ 1, a.ctx, abort_flag)) {
@@ -296,9 +318,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
         TileWalk w;
         w.start(a, it);
         int kt, klen;
+        long long koff;
         int8_t cls[2], ncls[2];
         bool any[2] = {false, false};
-        if (w.next(a, it, kt, klen, cls)) {
+        if (w.next(a, it, kt, klen, koff, cls)) {
           uint32_t kslot = ld % NSLOT, kph = (ld / NSLOT) & 1;
           uint32_t vslot = (ld + 1) % NSLOT, vph = ((ld + 1) / NSLOT) & 1;
           ld += 2;
@@ -312,7 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
           umma_commit(&slot_empty[kslot]);
           while (true) {
             int nkt, nklen;
-            const bool has_next = w.next(a, it, nkt, nklen, ncls);
+            long long nkoff;
+            const bool has_next = w.next(a, it, nkt, nklen, nkoff, ncls);
             uint32_t nkslot = 0, nkph = 0, nvslot = 0, nvph = 0;
             if (has_next) {
               nkslot = ld % NSLOT;
@@ -348,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
             if (!has_next) break;
             umma_commit(&slot_empty[nkslot]);
             kslot = nkslot; kph = nkph; vslot = nvslot; vph = nvph;
-            kt = nkt; klen = nklen;
+            kt = nkt; klen = nklen; koff = nkoff;
             cls[0] = ncls[0];
             cls[1] = ncls[1];
           }
@@ -378,12 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
     for (int round = 0; ok && item_at(a, round, it); ++round) {
       float m = -INFINITY, l = 0.f;
       bool any = false;
-      const long long q_pos = static_cast<long long>(a.q_offset) + it.q0[t] + row;
+      const long long st = pos_stride(a);
       TileWalk w;
       w.start(a, it);
       int kt, klen;
+      long long koff;
       int8_t cls[2];
-      while (w.next(a, it, kt, klen, cls)) {
+      while (w.next(a, it, kt, klen, koff, cls)) {
         if (cls[t] == kSkip) continue;
         if (!(ok = mbar_wait(&s_full[t], sph & 1, a.ctx, abort_flag))) break;
         ++sph;
@@ -401,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
         if (cls[t] == kPartial || klen < kBN) {
           long long lim = klen;
           if (a.causal) {
-            const long long vis = q_pos - (static_cast<long long>(a.k_offset) + kt) + 1;
+            const long long vis = visible_keys(it.q0[t] + row, kt, it.qoff, koff, st);
             lim = vis < lim ? vis : lim;
           }
 #pragma unroll
@@ -575,8 +600,9 @@ int dispatch(int dqk, int dv, const CUtensorMap& tq, const CUtensorMap& tk, cons
 }  // namespace
 
 int launch_tc_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
-                        int q_offset, int k_offset, int causal, float scale, void* out,
-                        bool out_f32, float* lse, const DeviceInfo& dev, cudaStream_t stream) {
+                        int q_offset, int k_offset, long long stride, int causal,
+                        int striped, float scale, void* out, bool out_f32, float* lse,
+                        const DeviceInfo& dev, cudaStream_t stream) {
   if (s.dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv;
   const uint64_t hq = static_cast<uint64_t>(s.B) * s.Hq;
@@ -598,6 +624,8 @@ int launch_tc_attention(const void* q, const void* k, const void* v, const ra_sh
   a.q_offset = q_offset;
   a.k_offset = k_offset;
   a.causal = causal;
+  a.striped = striped;
+  a.stride = striped ? P : stride;
   a.scale_log2 = scale * kLog2e;
   a.out = out;
   a.lse = lse;

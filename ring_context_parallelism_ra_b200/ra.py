@@ -17,7 +17,8 @@ import numpy as np
 import torch
 
 __all__ = [
-    "RAError", "library_path", "lib", "Shape", "block_partial", "lse_merge", "ring_forward",
+    "RAError", "library_path", "lib", "Shape", "block_partial", "block_partial_strided",
+    "lse_merge", "ring_forward", "ring_forward_striped",
     "ring_forward_host", "decode_workspace_bytes", "decode_partial", "decode_partial_noalloc",
     "decode_merge",
     "decode_pass_q", "block_class", "block_class_device", "get_status", "set_wait_limit_ns",
@@ -29,7 +30,8 @@ RA_F32, RA_BF16 = 0, 1
 
 # Every symbol include/ra.h declares.
 EXPORTED = (
-    "ra_block_partial", "ra_lse_merge", "ra_ring_forward", "ra_decode_workspace_bytes",
+    "ra_block_partial", "ra_block_partial_strided", "ra_lse_merge", "ra_ring_forward",
+    "ra_ring_forward_striped", "ra_decode_workspace_bytes",
     "ra_decode_partial", "ra_decode_partial_noalloc", "ra_decode_merge", "ra_block_class", "ra_block_class_device",
     "ra_get_status", "ra_set_wait_limit_ns", "ra_check_wait_timeout", "ra_status_string",
     "ra_launch_count", "ra_shutdown",
@@ -72,6 +74,8 @@ def lib() -> ctypes.CDLL:
         sp = ctypes.POINTER(Shape)
         sig = {
             "ra_block_partial": (i, [vp, vp, vp, sp, i, i, i, f, vp, vp, vp]),
+            "ra_block_partial_strided": (i, [vp, vp, vp, sp, i, i, i, i, f, vp, vp, vp]),
+            "ra_ring_forward_striped": (i, [vp, vp, vp, i, i, f, vp, vp, sp, vp]),
             "ra_lse_merge": (i, [vp, vp, i, sp, vp, i, vp, vp]),
             "ra_ring_forward": (i, [vp, vp, vp, i, i, f, vp, vp, sp, vp]),
             "ra_decode_workspace_bytes": (sz, [sp]),
@@ -151,6 +155,25 @@ def block_partial(q, k, v, q_offset=0, k_offset=0, causal=True, scale=None, o_pa
     return o_part, lse_part
 
 
+def block_partial_strided(q, k, v, q_offset, k_offset, pos_stride, causal=True, scale=None,
+                          o_part=None, lse_part=None, stream=None):
+    """Block partial with positions q_offset + t * pos_stride / k_offset + u * pos_stride
+    (the (i, j) block of a striped split is q_offset = i, k_offset = j, pos_stride = P)."""
+    s = _shape(q, k, v)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    if o_part is None:
+        o_part = torch.empty((s.B, s.Hq, s.n_q, s.d_v), device=q.device, dtype=torch.float32)
+    if lse_part is None:
+        lse_part = torch.empty((s.B, s.Hq, s.n_q), device=q.device, dtype=torch.float32)
+    rc = lib().ra_block_partial_strided(_need(q, "q"), _need(k, "k", q.dtype),
+                                        _need(v, "v", q.dtype), ctypes.byref(s), int(q_offset),
+                                        int(k_offset), int(pos_stride), int(bool(causal)),
+                                        float(scale), _need(o_part, "o_part", torch.float32),
+                                        _need(lse_part, "lse_part", torch.float32), _stream(stream))
+    _check("ra_block_partial_strided", rc)
+    return o_part, lse_part
+
+
 def lse_merge(o_parts, lse_parts, out_dtype=torch.float32, out=None, lse=None, stream=None,
               _name="ra_lse_merge"):
     """Merge P stacked partials o_parts [P,B,H,n,d_v], lse_parts [P,B,H,n]."""
@@ -182,6 +205,24 @@ def ring_forward(q, k, v, P, causal=True, scale=None, out=None, lse=None, stream
                                int(P), int(bool(causal)), float(scale), _need(out, "out", q.dtype),
                                _need(lse, "lse", torch.float32), ctypes.byref(s), _stream(stream))
     _check("ra_ring_forward", rc)
+    return out, lse
+
+
+def ring_forward_striped(q, k, v, P, causal=True, scale=None, out=None, lse=None, stream=None):
+    """Fused ring over a striped split: row i * (n / P) + r of q, k, v, out and
+    lse is token r * P + i."""
+    s = _shape(q, k, v)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    if out is None:
+        out = torch.empty((s.B, s.Hq, s.n_q, s.d_v), device=q.device, dtype=q.dtype)
+    if lse is None:
+        lse = torch.empty((s.B, s.Hq, s.n_q), device=q.device, dtype=torch.float32)
+    rc = lib().ra_ring_forward_striped(_need(q, "q"), _need(k, "k", q.dtype),
+                                       _need(v, "v", q.dtype), int(P), int(bool(causal)),
+                                       float(scale), _need(out, "out", q.dtype),
+                                       _need(lse, "lse", torch.float32), ctypes.byref(s),
+                                       _stream(stream))
+    _check("ra_ring_forward_striped", rc)
     return out, lse
 
 

@@ -26,7 +26,7 @@ from dataclasses import dataclass, field
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "workload", "draw_slice", "make_qkv",
-           "make_workload_inputs", "prefill_flops", "decode_kv_bytes"]
+           "make_workload_inputs", "prefill_flops", "decode_kv_bytes", "striped_order"]
 
 _TENSOR_ID = {"q": 1, "k": 2, "v": 3}
 
@@ -124,3 +124,15 @@ def decode_kv_bytes(wl: Workload) -> int:
     """Bytes of K and V one decode step must read (the whole cache, once)."""
     esz = 4 if wl.dtype == "f32" else 2
     return wl.B * wl.Hkv * wl.n * (wl.d_qk + wl.d_v) * esz
+
+
+def striped_order(n: int, P: int):
+    """Token order of a striped split: partition i holds tokens i, i + P,
+    i + 2P, ..., partitions stored one after another, so row i * (n / P) + r
+    holds token r * P + i.  Returns that token index for every row (a
+    permutation; ``x[:, :, order]`` lays a BHSD tensor out striped and
+    ``y[:, :, argsort(order)]`` restores token order)."""
+    if n % P:
+        raise ValueError("n must be divisible by P")
+    L = n // P
+    return [r * P + i for i in range(P) for r in range(L)]

@@ -97,3 +97,75 @@ def test_ring_order_is_receive_from_previous():
 def test_uneven_split_rejected():
     with pytest.raises(ValueError):
         partition_bounds(10, 4)
+
+
+# ---------------------------------------------------------- striped split --
+
+def _brute_positions(q, k, v, scale, qp, kp):
+    import math as m
+    nq, d = q.shape
+    nk = k.shape[0]
+    O = np.zeros((nq, v.shape[1]))
+    L = np.zeros(nq)
+    for t in range(nq):
+        vis = [u for u in range(nk) if kp[u] <= qp[t]]
+        if not vis:
+            L[t] = -np.inf
+            continue
+        s = {u: scale * m.fsum(q[t, c] * k[u, c] for c in range(d)) for u in vis}
+        mx = max(s.values())
+        lse = mx + m.log(m.fsum(m.exp(s[u] - mx) for u in vis))
+        L[t] = lse
+        for c in range(v.shape[1]):
+            O[t, c] = m.fsum(m.exp(s[u] - lse) * v[u, c] for u in vis)
+    return O, L
+
+
+def test_explicit_positions_match_brute_force():
+    from oracle.blockwise import striped_positions
+    rng = np.random.default_rng(60)
+    n, P = 12, 3
+    q = rng.standard_normal((1, 1, 4, 5))
+    k = rng.standard_normal((1, 1, 4, 5))
+    v = rng.standard_normal((1, 1, 4, 3))
+    for i in range(P):
+        for j in range(P):
+            qp, kp = striped_positions(n, P, i), striped_positions(n, P, j)
+            O, L = attention(q, k, v, 0.6, True, q_positions=qp, k_positions=kp)
+            Ob, Lb = _brute_positions(q[0, 0], k[0, 0], v[0, 0], 0.6, qp, kp)
+            fin = np.isfinite(Lb)
+            assert np.array_equal(np.isfinite(L[0, 0]), fin)
+            assert np.abs(O[0, 0] - Ob).max() <= 1e-12
+            assert np.abs(L[0, 0][fin] - Lb[fin]).max() <= 1e-12
+
+
+def test_striped_layout_is_a_permutation_of_full_attention():
+    from ring_context_parallelism_ra_b200.workloads import striped_order
+    rng = np.random.default_rng(61)
+    n, P = 24, 4
+    q = rng.standard_normal((1, 2, n, 6))
+    k = rng.standard_normal((1, 1, n, 6))
+    v = rng.standard_normal((1, 1, n, 4))
+    order = np.array(striped_order(n, P))
+    assert sorted(order.tolist()) == list(range(n))
+    assert order[1] == P and order[n // P] == 1          # row r of partition i is r*P + i
+    O, L = attention(q, k, v, 0.4, True)
+    Os, Ls = attention(q[:, :, order], k[:, :, order], v[:, :, order], 0.4, True,
+                       q_positions=order, k_positions=order)
+    assert np.abs(Os - O[:, :, order]).max() <= 1e-12
+    assert np.abs(Ls - L[:, :, order]).max() <= 1e-12
+
+
+def test_striped_blocks_are_balanced():
+    # contiguous split: block (i, j) has L^2, L(L+1)/2 or 0 visible pairs;
+    # striped split: L(L+1)/2 for j <= i and L(L-1)/2 for j > i (every block
+    # about half full, the page's reason for striping)
+    from oracle.blockwise import striped_block_visible
+    for n, P in [(16, 4), (48, 3), (64, 8)]:
+        L = n // P
+        for i in range(P):
+            for j in range(P):
+                want = L * (L + 1) // 2 if j <= i else L * (L - 1) // 2
+                assert striped_block_visible(n, P, i, j) == want
+        total = sum(striped_block_visible(n, P, i, j) for i in range(P) for j in range(P))
+        assert total == n * (n + 1) // 2
