@@ -274,6 +274,7 @@ def run_ours(args, world, rank):
     torch.cuda.empty_cache()
 
     decode = None if args.skip_decode else run_decode_leg(args, world, rank, peaks, peaks_kind)
+    striped = None if args.skip_striped else run_striped_leg(args, world, rank, workload(3), peaks)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -292,10 +293,86 @@ def run_ours(args, world, rank):
     }
     if decode is not None:
         line["decode"] = decode
+    if striped is not None:
+        line["striped"] = striped
     return line
 
 
 TC_FILES = ["tc_attention.cu", "ptx.cuh", "block_class.cuh"]
+
+
+def run_striped_leg(args, world, rank, wl, peaks):
+    """Striped split (token p in partition p mod P) on workload `wl` (the
+    causal GQA 128K workload, P = 8, where one partition block alone fills
+    the GPU, so a block's time tracks its work):
+    (a) the fused striped ring vs the fused contiguous ring, TFLOP/s;
+    (b) P devices emulated one after another: device i runs its ring steps as
+        block partials (Q_i against each KV_j it must see), timed as one chain
+        of launches; the slowest device bounds a real ring's time.  Contiguous
+        devices skip their fully masked blocks, striped devices have none."""
+    from ring_context_parallelism_ra_b200.workloads import striped_order
+    dev = torch.device("cuda")
+    q, k, v = make_workload_inputs(dataclasses.replace(wl, seed=wl.seed + 1000 * rank), device=dev)
+    flops = prefill_flops(wl)
+    n, P, L = wl.n, wl.P, wl.n // wl.P
+    order = torch.tensor(striped_order(n, P), device=dev)
+    qs, ks, vs = (x[:, :, order].contiguous() for x in (q, k, v))
+    out = torch.empty((wl.B, wl.Hq, n, wl.d_v), device=dev, dtype=wl.torch_dtype)
+    lse = torch.empty((wl.B, wl.Hq, n), device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    steps = 3
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    ms_striped = timed(lambda: ra.ring_forward_striped(qs, ks, vs, P, wl.causal, wl.scale, out, lse))
+    ms_contig = timed(lambda: ra.ring_forward(q, k, v, P, wl.causal, wl.scale, out, lse))
+    parts = {}
+    for name, (qq, kk, vv) in (("contiguous", (q, k, v)), ("striped", (qs, ks, vs))):
+        qi = [qq[:, :, i * L:(i + 1) * L].contiguous() for i in range(P)]
+        kj = [kk[:, :, j * L:(j + 1) * L].contiguous() for j in range(P)]
+        vj = [vv[:, :, j * L:(j + 1) * L].contiguous() for j in range(P)]
+        o = torch.empty((wl.B, wl.Hq, L, wl.d_v), device=dev)
+        ll = torch.empty((wl.B, wl.Hq, L), device=dev)
+        per_dev = []
+        for i in range(P):
+            if name == "contiguous":
+                blocks = [(j, i * L, j * L, 1) for j in range(P) if not (wl.causal and j > i)]
+            else:
+                blocks = [(j, i, j, P) for j in range(P)]
+
+            def chain(blocks=blocks, i=i):
+                for j, qo, ko, st in blocks:
+                    ra.block_partial_strided(qi[i], kj[j], vj[j], qo, ko, st, wl.causal, wl.scale, o, ll)
+            per_dev.append(timed(chain))
+        parts[name] = per_dev
+    assert ra.get_status() == ra.RA_OK
+    res = {"workload": wl.name,
+           "fused_striped_tflops": round(flops / (ms_striped * 1e-3) / 1e12, 2),
+           "fused_contiguous_tflops": round(flops / (ms_contig * 1e-3) / 1e12, 2),
+           "emulated_devices": P,
+           "device_ms_contiguous": [round(x, 4) for x in parts["contiguous"]],
+           "device_ms_striped": [round(x, 4) for x in parts["striped"]],
+           "slowest_device_ms": {k: round(max(v), 4) for k, v in parts.items()},
+           "ring_speedup_striped_over_contiguous":
+               round(max(parts["contiguous"]) / max(parts["striped"]), 3),
+           "note": "block partials per emulated device, one device at a time on this GPU"}
+    del q, k, v, qs, ks, vs, out, lse, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_decode_leg(args, world, rank, peaks, peaks_kind):
@@ -379,6 +456,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 5])
     ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-striped", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:

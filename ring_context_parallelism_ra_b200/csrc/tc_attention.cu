@@ -116,7 +116,18 @@ __device__ __forceinline__ bool item_at(const TcArgs& a, int round, Item& it) {
   const int bhs = a.B * a.Hq;
   const int r = static_cast<int>(idx / bhs);
   it.bh = static_cast<int>(idx % bhs);
-  const int tp = a.causal ? (a.n_pairs - 1 - r) : r;  // heaviest pairs first when causal
+  // heaviest pairs first when causal: work grows with the row's token
+  // position, i.e. with the pair index (contiguous) or with the pair index
+  // inside its partition (striped, all partitions' pairs of one index together)
+  int tp = r;
+  if (a.causal) {
+    if (a.striped) {
+      const int pp = a.n_pairs / a.P;  // pairs per partition (n / P % 256 == 0)
+      tp = (r % a.P) * pp + (pp - 1 - r / a.P);
+    } else {
+      tp = a.n_pairs - 1 - r;
+    }
+  }
   it.b = it.bh / a.Hq;
   it.g = (it.bh % a.Hq) / (a.Hq / a.Hkv);
   for (int t = 0; t < 2; ++t) {
