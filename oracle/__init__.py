@@ -24,6 +24,8 @@ Modules:
                      only to pin the definition against the method's invariants.
 * ``merge``       -- N-way (O, LSE) merge of normalised partials.
 * ``block_class`` -- SKIP / PARTIAL / FULL per tile from the explicit mask.
+* ``backward``    -- the gradients dQ, dK, dV of the definition (chain rule),
+                     whole-row and block by block in ring order.
 * ``costs``       -- FLOP / byte formulas of the pages.
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against brute

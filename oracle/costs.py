@@ -7,7 +7,7 @@ and that these reproduce the pages' worked numbers.
 from __future__ import annotations
 
 __all__ = ["kv_cache_bytes", "decode_latency_lower_bound_s", "prefill_flops",
-           "pass_kv_bytes_per_chip", "kv_bytes_per_chip", "mla_ckv_bytes"]
+           "backward_flops", "pass_kv_bytes_per_chip", "kv_bytes_per_chip", "mla_ckv_bytes"]
 
 
 def kv_cache_bytes(L, h_kv, d_h, n, b):
@@ -28,6 +28,16 @@ def prefill_flops(B, S, d_qk, d_v, heads=1, causal=False):
     formula counts one head and the full square; ``heads`` multiplies it and
     ``causal`` halves it (the causal triangle, 1/2 rather than (n+1)/(2n))."""
     f = 2 * B * S * S * (d_qk + d_v) * heads
+    return f // 2 if causal else f
+
+
+def backward_flops(B, S, d_qk, d_v, heads=1, causal=False):
+    """Algorithmic FLOPs of the attention backward pass (the pages give none):
+    the five products of its definition, each 2 S^2 times its inner size --
+    scores recomputed (D_qk), dP = dO V^T (D_v), dV = P^T dO (D_v),
+    dQ = dS K (D_qk), dK = dS^T Q (D_qk).  Causal halves it, as for
+    ``prefill_flops``."""
+    f = 2 * B * S * S * (3 * d_qk + 2 * d_v) * heads
     return f // 2 if causal else f
 
 
