@@ -275,6 +275,10 @@ def run_ours(args, world, rank):
 
     decode = None if args.skip_decode else run_decode_leg(args, world, rank, peaks, peaks_kind)
     striped = None if args.skip_striped else run_striped_leg(args, world, rank, workload(3), peaks)
+    backward = None
+    if not args.skip_backward and wl.dtype == "bf16":
+        backward = [run_backward_leg(args, world, rank, w, peaks, peaks_kind)
+                    for w in (wl, workload(3))]
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -295,7 +299,65 @@ def run_ours(args, world, rank):
         line["decode"] = decode
     if striped is not None:
         line["striped"] = striped
+    if backward is not None:
+        line["backward"] = backward
     return line
+
+
+def run_backward_leg(args, world, rank, wl, peaks, peaks_kind):
+    """Gradients of the fused ring (dQ, dK, dV from the forward's O, LSE and a
+    random dO) on workload `wl`: TFLOP/s of the whole backward call (row
+    statistics, the tensor-core kernel, the dQ conversion), L2 flushed
+    between steps."""
+    from ring_context_parallelism_ra_b200.workloads import backward_flops, make_dout
+    dev = torch.device("cuda")
+    wr = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
+    q, k, v = make_workload_inputs(wr, device=dev)
+    g = make_dout(wl.B, wl.Hq, wl.n, wl.d_v, wl.torch_dtype, seed=wr.seed, device=dev)
+    out, lse = ra.ring_forward(q, k, v, wl.P, wl.causal, wl.scale)
+    ws = torch.empty(ra.backward_workspace_bytes(q, k, v), dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ra.ring_backward(q, k, v, out, lse, g, wl.P, wl.causal, wl.scale, dq, dk, dv, ws)
+
+    for _ in range(3):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    launches0 = ra.launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for s, e in ev:
+            flush.zero_()
+            s.record(stream)
+            step()
+            e.record(stream)
+        torch.cuda.synchronize()
+    launches = ra.launch_count() - launches0
+    assert ra.get_status() == ra.RA_OK
+    ms_local = statistics.mean(s.elapsed_time(e) for s, e in ev)
+    ms = max_over_ranks(ms_local, world)
+    flops = backward_flops(wl)
+    achieved = flops / (ms_local * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    del q, k, v, g, out, lse, ws, dq, dk, dv, flush
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "value": round(world * flops / (ms * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "flops_per_step": flops,
+            "flop_convention": "2*B*Hq*n^2*(3*d_qk+2*d_v), x1/2 causal",
+            "launches_per_step": launches // steps,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "peak_kind": f"{peaks_kind} bf16 burst",
+                         "kernel": "ring_backward (prep + tcgen05 kernel + dQ conversion)"},
+            "clocks": clk.summary()}
 
 
 TC_FILES = ["tc_attention.cu", "ptx.cuh", "block_class.cuh"]
@@ -457,6 +519,7 @@ def main():
     ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 5])
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-striped", action="store_true")
+    ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:

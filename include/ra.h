@@ -216,6 +216,93 @@ int ra_decode_merge(const float* o_parts, const float* lse_parts, int P, const r
                     void* out, ra_dtype out_dtype, float* lse, void* stream);
 
 /*
+ * Backward pass.  The pages name it (page "AI 推理系列（十一）：Ring Attention
+ * 如何让多张 GPU 共同计算一条超长序列": training keeps what the backward pass
+ * needs, and its data dependencies across blocks are a place to look when
+ * results go wrong) but give no algorithm; the gradients below are the chain
+ * rule of the forward definition (page "长上下文的第一性挑战", Eq.
+ * (lc-ch-attention)) for a loss that depends on O through dO:
+ *   P = exp(scale Q K^T - LSE) on visible pairs (the forward's final LSE),
+ *   dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P (dP - D),
+ *   dQ = scale dS K,  dK = scale dS^T Q,
+ * with dK, dV of a KV head summed over the query heads of its group.  In the
+ * ring, KV_j travels with its accumulators dK_j, dV_j and collects one share
+ * per query partition while dQ_i collects at its partition.
+ * Supported head dims (bf16 and fp32): d_qk, d_v in {64, 128}.
+ */
+
+/*
+ * ra_backward_workspace_bytes -- device workspace the backward calls need for
+ * `shape` (an fp32 dQ accumulator and two row vectors, padded to 128 rows
+ * per head): about B * Hq * n_q * (d_qk + 2) * 4 bytes.  0 on invalid shape.
+ */
+size_t ra_backward_workspace_bytes(const ra_shape* shape);
+
+/*
+ * ra_backward_delta -- D = rowsum(dO * O) per query row.
+ *   out, dout   : device [B, Hq, n_q, d_v] of shape->dtype (O of the forward
+ *                 and the gradient arriving at it).
+ *   delta       : device fp32 [B, Hq, n_q].
+ * Errors: RA_ERR_INVALID, RA_ERR_CUDA.
+ */
+int ra_backward_delta(const void* out, const void* dout, const ra_shape* shape, float* delta,
+                      void* stream);
+
+/*
+ * ra_ring_backward -- gradients of ra_ring_forward for all P partitions of
+ * one sequence: dQ, dK, dV of q, k, v.  Each key tile of KV_j meets the query
+ * partitions in ring order j, j+1, ... (mod P), fully masked tiles skipped;
+ * its dK, dV stay on chip for the whole walk.
+ *   q, k, v     : as ra_ring_forward (n_q == n_k == n, n % P == 0).
+ *   out, lse    : the forward's outputs for these inputs ([B, Hq, n, d_v] of
+ *                 the input dtype; fp32 [B, Hq, n]).
+ *   dout        : device [B, Hq, n, d_v], input dtype.
+ *   dq, dk, dv  : device outputs of the input dtype, shaped like q, k, v.
+ *   workspace   : device, >= ra_backward_workspace_bytes(shape), 16-B
+ *                 aligned, owned by the caller; contents on entry ignored.
+ * Errors: RA_ERR_INVALID (shapes, null, misaligned, workspace too small),
+ * RA_ERR_UNSUPPORTED (head dims), RA_ERR_CUDA.  bf16 runs on the tensor
+ * cores; fp32 in exact fp32 arithmetic.
+ */
+int ra_ring_backward(const void* q, const void* k, const void* v, const void* out,
+                     const float* lse, const void* dout, int P, int causal, float scale, void* dq,
+                     void* dk, void* dv, const ra_shape* shape, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
+ * ra_ring_backward_striped -- the same over the striped split of
+ * ra_ring_forward_striped (tensor row R = i * (n / P) + r is token r * P + i;
+ * gradients in the same row order).  Needs (n / P) % 128 == 0, else
+ * RA_ERR_UNSUPPORTED.
+ */
+int ra_ring_backward_striped(const void* q, const void* k, const void* v, const void* out,
+                             const float* lse, const void* dout, int P, int causal, float scale,
+                             void* dq, void* dk, void* dv, const ra_shape* shape, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * ra_block_backward -- one (Q range, KV range) block's share of the
+ * gradients, added into fp32 accumulators: the step a device of the ring
+ * takes when KV_j (with dK_j, dV_j) reaches Q_i.  P is formed against the
+ * FINAL row statistics, so shares of different blocks simply add up.
+ *   q, k, v, dout : device, shapes as ra_block_partial (dout [B, Hq, n_q, d_v]).
+ *   lse           : device fp32 [B, Hq, n_q], the forward's final LSE of
+ *                   these rows (over all keys, not just this block).
+ *   delta         : device fp32 [B, Hq, n_q], from ra_backward_delta.
+ *   q_offset, k_offset, pos_stride, causal : positions as
+ *                   ra_block_partial_strided.
+ *   dq_acc        : device fp32 [B, Hq, n_q, d_qk], += this block's dQ share.
+ *   dk_acc, dv_acc: device fp32 [B, Hkv, n_k, d_qk / d_v], += shares.
+ *   workspace     : as ra_ring_backward.
+ * Errors: as ra_ring_backward.
+ */
+int ra_block_backward(const void* q, const void* k, const void* v, const void* dout,
+                      const float* lse, const float* delta, const ra_shape* shape, int q_offset,
+                      int k_offset, int pos_stride, int causal, float scale, float* dq_acc,
+                      float* dk_acc, float* dv_acc, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
  * ra_block_class -- causal class of every (query block, key block) pair,
  * host side: 0 = SKIP (no visible pair), 1 = PARTIAL, 2 = FULL (every pair
  * visible).  Blocks at the ragged end cover only existing rows / keys.  With
@@ -239,7 +326,8 @@ int ra_block_class_device(int n_q, int n_k, int q_block, int k_block, int q_offs
  * ra_get_status -- synchronise `stream`, then read and clear the current
  * device's status word.  Returns RA_OK, or RA_ERR_TIMEOUT if a kernel's
  * bounded wait expired since the last call (its results are then invalid),
- * or RA_ERR_CUDA if the synchronisation itself failed.
+ * or RA_ERR_CUDA if the synchronisation itself failed or a kernel could not
+ * align its shared-memory tiles and returned without computing.
  */
 int ra_get_status(void* stream);
 

@@ -40,7 +40,8 @@ import numpy as np
 from .attention import _as_f64, attention, gqa_group
 from .blockwise import partition_bounds, ring_order
 
-__all__ = ["attention_backward", "ring_attention_backward", "row_delta"]
+__all__ = ["attention_backward", "attention_backward_sampled", "ring_attention_backward",
+           "row_delta"]
 
 
 def _positions(n, offset, positions):
@@ -96,6 +97,66 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, q_offset: int = 
                 dv[b, g] += p.T @ doh[r]
                 dq[b, h, r] = scale * (ds @ kk)
                 dk[b, g] += scale * (ds.T @ qh[r])
+    return dq, dk, dv
+
+
+def attention_backward_sampled(q, k, v, do, scale: float, causal: bool, rows, keys,
+                               heads=None, kv_heads=None, row_chunk: int = 2048):
+    """The same gradients at a sample: dQ at query ``rows`` of query ``heads``,
+    dK and dV at ``keys`` of ``kv_heads`` (positions 0..n-1, n_q == n_k).
+
+    dQ_t needs only row t; dK_u, dV_u need column u of every row, i.e. every
+    row's LSE and D, which come from ``oracle.attention.attention`` over all
+    rows.  Returns dq [B, len(heads), len(rows), dqk],
+    dk [B, len(kv_heads), len(keys), dqk], dv [B, len(kv_heads), len(keys), dv].
+    """
+    B, h_q, n, dqk = q.shape
+    h_kv = k.shape[1]
+    dvd = v.shape[-1]
+    grp = gqa_group(h_q, h_kv)
+    rows = np.asarray(rows, dtype=np.int64)
+    keys = np.asarray(keys, dtype=np.int64)
+    heads = list(range(h_q)) if heads is None else list(heads)
+    kv_heads = list(range(h_kv)) if kv_heads is None else list(kv_heads)
+    pos = np.arange(n, dtype=np.int64)
+    dq = np.zeros((B, len(heads), len(rows), dqk))
+    dk = np.zeros((B, len(kv_heads), len(keys), dqk))
+    dv = np.zeros((B, len(kv_heads), len(keys), dvd))
+    need_all = sorted(set(heads) | {g * grp + r for g in kv_heads for r in range(grp)})
+    for b in range(B):
+        stats = {}
+        for h in need_all:
+            o, lse = attention(q[b:b + 1], k[b:b + 1], v[b:b + 1], scale, causal,
+                               heads=[h], row_chunk=row_chunk)
+            stats[h] = (lse[0, 0], (o[0, 0] * _as_f64(do[b, h])).sum(axis=1))
+        for hi, h in enumerate(heads):
+            g = h // grp
+            kk, vv = _as_f64(k[b, g]), _as_f64(v[b, g])
+            qr, dor = _as_f64(q[b, h][rows]), _as_f64(do[b, h][rows])
+            lse, dlt = stats[h][0][rows], stats[h][1][rows]
+            s = (qr @ kk.T) * scale
+            if causal:
+                s = np.where(pos[None, :] <= rows[:, None], s, -np.inf)
+            live = np.isfinite(lse)
+            p = np.zeros_like(s)
+            p[live] = np.exp(s[live] - lse[live, None])
+            ds = p * (dor @ vv.T - dlt[:, None])
+            dq[b, hi] = scale * (ds @ kk)
+        for gi, g in enumerate(kv_heads):
+            kc, vc = _as_f64(k[b, g][keys]), _as_f64(v[b, g][keys])
+            for r in range(grp):
+                h = g * grp + r
+                qa, doa = _as_f64(q[b, h]), _as_f64(do[b, h])
+                lse, dlt = stats[h]
+                st = (qa @ kc.T) * scale                      # [n, len(keys)]
+                if causal:
+                    st = np.where(keys[None, :] <= pos[:, None], st, -np.inf)
+                live = np.isfinite(lse)
+                p = np.zeros_like(st)
+                p[live] = np.exp(st[live] - lse[live, None])
+                ds = p * (doa @ vc.T - dlt[:, None])
+                dk[b, gi] += scale * (ds.T @ qa)
+                dv[b, gi] += p.T @ doa
     return dq, dk, dv
 
 

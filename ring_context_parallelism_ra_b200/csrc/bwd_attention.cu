@@ -1,0 +1,775 @@
+// Backward pass of exact attention on the tensor cores (bf16 inputs), plus the
+// small kernels around it (row statistics in, dQ out) shared with the fp32
+// path.  What is computed is stated in bwd.cuh.
+//
+// CTA layout of the tensor-core kernel (384 threads, one CTA per SM,
+// persistent; work item = one 128-key tile of one (batch, KV head)):
+//   warp 0      TMA producer: K, V of the item; then per visit Q, dO (TMA) and
+//               the visit's -LSE log2(e) and D vectors (bulk copies), two stages
+//   warp 1      tcgen05.mma issuer; owns the tensor-memory allocation
+//   warps 2-3   idle
+//   warps 4-7   "compute": thread r owns key r of the tile (TMEM lane r):
+//               P^T = 2^(scale log2(e) S^T - LSE log2(e)) into TMEM as bf16,
+//               then dS^T = P^T (dP^T - D) into shared memory as bf16
+//   warps 8-11  "reduce": reads each visit's dQ tile out of TMEM and adds it
+//               into the fp32 workspace (red.add, a warp covers 32 consecutive
+//               floats); at the end of the item writes dK, dV
+// Registers: launched at 168 per thread; setmaxnreg moves them to 224
+// (compute) + 160 (reduce) + 120 (producer / MMA warpgroup) = 504 = 3 x 168.
+//
+// Per visit (query tile t of head h against the item's key tile):
+//   S^T  = K Q_t^T        M = 128 keys, N = 128 queries   (A, B K-major)
+//   dP^T = V dO_t^T       M = 128 keys, N = 128 queries   (A, B K-major)
+//   dV  += P^T dO_t       A = P^T in TMEM, B = dO_t MN-major
+//   dK  += dS^T Q_t       A = dS^T K-major, B = Q_t MN-major
+//   dQ_t = dS K           A = the same dS bytes read MN-major, B = K MN-major
+// The dS tile is written once: its rows (keys) of 64 query columns in
+// 128-byte-swizzled atoms are at the same time the K-major layout of dS^T and
+// the MN-major layout of dS.
+//
+// Tensor memory (512 columns): S^T [0,128) (P^T packed over its first 64
+// columns), dP^T [128,256), dV [256,256+DV), dK [256+DV,256+DV+DQK), dQ in its
+// own columns after dK when they fit (DQK = DV = 64, or DQK = 64, DV = 128),
+// else over the S^T columns once dV has read P^T (MMAs of one thread execute
+// in issue order; the next S^T waits until dQ has been read out).
+#include <cuda.h>
+
+#include "block_class.cuh"
+#include "bwd.cuh"
+#include "common.cuh"
+#include "launch.h"
+#include "ptx.cuh"
+#include "tmap.h"
+
+namespace ra {
+
+namespace {
+
+constexpr int kT = 128;
+constexpr int kBox = 128 * 64 * 2;  // TMA box: 128 rows x 64 bf16
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsCompute = 224;
+constexpr int kRegsReduce = 160;
+constexpr int kRegsOther = 120;
+static_assert(kRegsCompute + kRegsReduce + kRegsOther <= 3 * kRegsLaunch,
+              "register split must fit the launch allocation");
+// setmaxnreg.inc may only raise a warpgroup's count and .dec only lower it.
+static_assert(kRegsCompute >= kRegsLaunch, "compute warpgroup grows (setmaxnreg.inc)");
+static_assert(kRegsReduce <= kRegsLaunch && kRegsOther <= kRegsLaunch,
+              "reduce and producer / MMA warpgroups shrink (setmaxnreg.dec)");
+constexpr int kSmemLimit = 232448;
+
+template <int DQK, int DV>
+struct BCfg {
+  static constexpr int QB = DQK / 64;
+  static constexpr int VB = DV / 64;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + QB * kBox;
+  static constexpr int Q_OFF = V_OFF + VB * kBox;      // two stages
+  static constexpr int DO_OFF = Q_OFF + 2 * QB * kBox;  // two stages
+  static constexpr int DS_OFF = DO_OFF + 2 * VB * kBox;
+  static constexpr int VEC_OFF = DS_OFF + 2 * kBox;     // [stage][-LSE log2e | D][128]
+  static constexpr int BAR_OFF = VEC_OFF + 2 * 2 * kT * 4;
+  static constexpr int USED = BAR_OFF + 256;
+  static_assert(USED <= kSmemLimit, "shared memory budget");
+  // Room left for aligning the dynamic shared memory base to 1024 bytes.
+  static constexpr int SMEM = USED + 1024 <= kSmemLimit ? USED + 1024 : kSmemLimit;
+  static constexpr int S_COL = 0;
+  static constexpr int DP_COL = 128;
+  static constexpr int DV_COL = 256;
+  static constexpr int DK_COL = 256 + DV;
+  static constexpr bool DQ_OWN = 256 + DV + 2 * DQK <= 512;
+  static constexpr int DQ_COL = DQ_OWN ? 256 + DV + DQK : S_COL;
+  static_assert(DQ_OWN || DQK <= 128, "dQ must fit over the S^T columns");
+  static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t ID_DV = idesc_bf16_f32(128, DV, 0, 1);
+  static constexpr uint32_t ID_DK = idesc_bf16_f32(128, DQK, 0, 1);
+  static constexpr uint32_t ID_DQ = idesc_bf16_f32(128, DQK, 1, 1);
+};
+
+// Bulk (non-tensor) copy global -> shared, completion as transaction bytes on
+// `bar`.  Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (the tensor cores read dS from shared memory).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Descriptors of successive K steps differ only in the start address field.
+// K-major operand: a K step of 16 bf16 is 32 bytes inside a 64-wide atom,
+// atoms (128 rows each) are kBox apart.  MN-major operand: a K step is 16
+// rows of 128 bytes = 2048 bytes.
+__device__ __forceinline__ uint32_t kmaj_step(int ks) {
+  return static_cast<uint32_t>(((ks >> 2) * kBox + (ks & 3) * 32) >> 4);
+}
+__device__ __forceinline__ uint32_t mnmaj_step(int ks) {
+  return static_cast<uint32_t>((ks * 2048) >> 4);
+}
+
+// D[128 x 128] = A B^T, A and B K-major with KD columns (S^T, dP^T).
+template <int KD>
+__device__ __forceinline__ void mma_kk(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc) {
+  const uint64_t da = sdesc_k_sw128(a), db = sdesc_k_sw128(b);
+#pragma unroll
+  for (int ks = 0; ks < KD / 16; ++ks)
+    umma_ss(d, da + kmaj_step(ks), db + kmaj_step(ks), idesc, ks > 0 ? 1u : 0u);
+}
+
+// dV (+)= P^T dO: A from tensor memory (128 queries = 64 packed columns).
+__device__ __forceinline__ void mma_tm(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t idesc,
+                                       bool acc) {
+  const uint64_t db = sdesc_mn_sw128(b, kBox);
+#pragma unroll
+  for (int ks = 0; ks < kT / 16; ++ks)
+    umma_ts(d, a_tmem + ks * 8, db + mnmaj_step(ks), idesc, (acc || ks > 0) ? 1u : 0u);
+}
+
+// dK (+)= dS^T Q: A K-major (keys x queries), B MN-major (queries x DQK).
+__device__ __forceinline__ void mma_km(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc,
+                                       bool acc) {
+  const uint64_t da = sdesc_k_sw128(a), db = sdesc_mn_sw128(b, kBox);
+#pragma unroll
+  for (int ks = 0; ks < kT / 16; ++ks)
+    umma_ss(d, da + kmaj_step(ks), db + mnmaj_step(ks), idesc, (acc || ks > 0) ? 1u : 0u);
+}
+
+// dQ = dS K: A MN-major (queries along M, keys along K), B MN-major (keys x DQK).
+__device__ __forceinline__ void mma_mm(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc) {
+  const uint64_t da = sdesc_mn_sw128(a, kBox), db = sdesc_mn_sw128(b, kBox);
+#pragma unroll
+  for (int ks = 0; ks < kT / 16; ++ks)
+    umma_ss(d, da + mnmaj_step(ks), db + mnmaj_step(ks), idesc, ks > 0 ? 1u : 0u);
+}
+
+// dK or dV of the item's keys out of tensor memory: `mul` times the
+// accumulator, stored (ring: bf16) or added (block: fp32).  Warp-collective.
+template <int D>
+__device__ __forceinline__ void store_key_grad(uint32_t taddr, bool any, bool valid, float mul,
+                                               void* dst, long long krow, int block_mode) {
+#pragma unroll
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    float o[32];
+    if (any) {
+      tmem_ld32f(taddr + c0, o);
+      tmem_ld_wait();
+      reg_fence32(o);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) o[c] = 0.f;
+    }
+    if (valid && block_mode) {
+      float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + krow * D + c0);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float4 x = d4[c];
+        x.x += o[4 * c] * mul;
+        x.y += o[4 * c + 1] * mul;
+        x.z += o[4 * c + 2] * mul;
+        x.w += o[4 * c + 3] * mul;
+        d4[c] = x;
+      }
+    } else if (valid) {
+      uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + krow * D + c0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        d4[c] = make_uint4(pack_bf16x2(o[8 * c] * mul, o[8 * c + 1] * mul),
+                           pack_bf16x2(o[8 * c + 2] * mul, o[8 * c + 3] * mul),
+                           pack_bf16x2(o[8 * c + 4] * mul, o[8 * c + 5] * mul),
+                           pack_bf16x2(o[8 * c + 6] * mul, o[8 * c + 7] * mul));
+    }
+  }
+}
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    BwdArgs a) {
+  using C = BCfg<DQK, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (pad > static_cast<uint32_t>(C::SMEM - C::USED)) {  // cannot align the tiles: report
+    if (threadIdx.x == 0) atomicExch(a.ctx.status, static_cast<int>(RA_ERR_CUDA));
+    return;
+  }
+  uint8_t* sm = smem_raw + pad;
+  uint8_t* sK = sm + C::K_OFF;
+  uint8_t* sV = sm + C::V_OFF;
+  uint8_t* sQ = sm + C::Q_OFF;
+  uint8_t* sdO = sm + C::DO_OFF;
+  uint8_t* sdS = sm + C::DS_OFF;
+  float* vec = reinterpret_cast<float*>(sm + C::VEC_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::BAR_OFF);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* q_full = bars + 2;   // [2]
+  uint64_t* q_empty = bars + 4;  // [2]
+  uint64_t* s_full = bars + 6;
+  uint64_t* dp_full = bars + 7;
+  uint64_t* p_full = bars + 8;
+  uint64_t* ds_full = bars + 9;
+  uint64_t* dq_full = bars + 10;
+  uint64_t* dq_empty = bars + 11;
+  uint64_t* acc_full = bars + 12;
+  uint64_t* acc_empty = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* kv_issued = abort_flag + 1;
+  volatile int* q_issued = abort_flag + 2;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, kT);
+    mbar_init(ds_full, kT);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, kT);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kT);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *kv_issued = 0;
+    *q_issued = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp < 4) regs_dec<kRegsOther>();
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      uint32_t nkv = 0, nq = 0;
+      BItem it;
+      bool ok = true;
+      for (int round = 0; ok && !*abort_flag && bwd_item_at(a, round, it); ++round) {
+        QWalk w;
+        w.start(a, it);
+        int qt, h;
+        if (!w.next(a, it, qt, h)) continue;
+        if (!(ok = mbar_wait(kv_empty, (nkv & 1) ^ 1, a.ctx, abort_flag))) break;
+        mbar_arrive_expect_tx(kv_full, (C::QB + C::VB) * kBox);
+        for (int bx = 0; bx < C::QB; ++bx)
+          tma_load_3d(sK + bx * kBox, &tm_k, kv_full, bx * 64, it.k0, it.bkv);
+        for (int bx = 0; bx < C::VB; ++bx)
+          tma_load_3d(sV + bx * kBox, &tm_v, kv_full, bx * 64, it.k0, it.bkv);
+        *kv_issued = static_cast<int>(++nkv);
+        do {
+          const int st = nq & 1;
+          if (!(ok = mbar_wait(&q_empty[st], ((nq >> 1) & 1) ^ 1, a.ctx, abort_flag))) break;
+          const int bh = it.b * a.Hq + h;
+          mbar_arrive_expect_tx(&q_full[st], (C::QB + C::VB) * kBox + 2 * kT * 4);
+          for (int bx = 0; bx < C::QB; ++bx)
+            tma_load_3d(sQ + (st * C::QB + bx) * kBox, &tm_q, &q_full[st], bx * 64, qt * kT, bh);
+          for (int bx = 0; bx < C::VB; ++bx)
+            tma_load_3d(sdO + (st * C::VB + bx) * kBox, &tm_do, &q_full[st], bx * 64, qt * kT,
+                        bh);
+          const long long vrow = (static_cast<long long>(bh) * a.ntq_ws + qt) * kT;
+          bulk_load(vec + st * 2 * kT, a.ws_nl2 + vrow, kT * 4, &q_full[st]);
+          bulk_load(vec + st * 2 * kT + kT, a.ws_d + vrow, kT * 4, &q_full[st]);
+          *q_issued = static_cast<int>(++nq);
+        } while (w.next(a, it, qt, h));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      uint32_t nkv = 0, nq = 0, nv = 0, nacc = 0;
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ);
+      const uint32_t adO = smem_u32(sdO), adS = smem_u32(sdS);
+      BItem it;
+      bool ok = true;
+      for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
+        QWalk w;
+        w.start(a, it);
+        int qt, h;
+        bool has = w.next(a, it, qt, h);
+        if (!has) continue;
+        if (!(ok = mbar_wait(kv_full, nkv & 1, a.ctx, abort_flag))) break;
+        ++nkv;
+        tc_fence_after();
+        bool first = true;
+        while (has) {
+          int nqt, nh;
+          const bool has_next = w.next(a, it, nqt, nh);
+          const int st = nq & 1;
+          if (!(ok = mbar_wait(&q_full[st], (nq >> 1) & 1, a.ctx, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t q_s = aQ + st * C::QB * kBox;
+          const uint32_t do_s = adO + st * C::VB * kBox;
+          if (!C::DQ_OWN) {  // S^T overwrites the previous dQ: wait until it is read out
+            if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
+            tc_fence_after();
+          }
+          mma_kk<DQK>(tmem + C::S_COL, aK, q_s, C::ID_S);
+          umma_commit(s_full);
+          mma_kk<DV>(tmem + C::DP_COL, aV, do_s, C::ID_S);
+          umma_commit(dp_full);
+          if (!(ok = mbar_wait(p_full, nv & 1, a.ctx, abort_flag))) break;
+          tc_fence_after();
+          if (first) {  // the previous item's dK, dV have been read out
+            if (!(ok = mbar_wait(acc_empty, (nacc & 1) ^ 1, a.ctx, abort_flag))) break;
+            tc_fence_after();
+          }
+          mma_tm(tmem + C::DV_COL, tmem + C::S_COL, do_s, C::ID_DV, !first);
+          if (!(ok = mbar_wait(ds_full, nv & 1, a.ctx, abort_flag))) break;
+          tc_fence_after();
+          mma_km(tmem + C::DK_COL, adS, q_s, C::ID_DK, !first);
+          if (C::DQ_OWN) {
+            if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
+            tc_fence_after();
+          }
+          mma_mm(tmem + C::DQ_COL, adS, aK, C::ID_DQ);
+          umma_commit(dq_full);
+          umma_commit(&q_empty[st]);
+          ++nq;
+          ++nv;
+          first = false;
+          if (!has_next) {
+            umma_commit(acc_full);
+            umma_commit(kv_empty);
+            ++nacc;
+          }
+          qt = nqt;
+          h = nh;
+          has = has_next;
+        }
+        if (!ok) break;
+      }
+      // every MMA issued so far has finished before the allocation goes away
+      umma_commit(drain);
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < a.ctx.wait_ns) {
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------- compute: P^T and dS^T --
+    regs_inc<kRegsCompute>();
+    const int row = threadIdx.x & 127;  // key of the tile = TMEM lane
+    const uint32_t lb = tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+    uint8_t* ds_row = sdS + row * 128;
+    const uint32_t sw = row & 7;
+    uint32_t nq = 0, nv = 0;
+    BItem it;
+    bool ok = true;
+    for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
+      QWalk w;
+      w.start(a, it);
+      int qt, h;
+      while (w.next(a, it, qt, h)) {
+        const int st = nq & 1;
+        if (!(ok = mbar_wait(&q_full[st], (nq >> 1) & 1, a.ctx, abort_flag))) break;
+        if (!(ok = mbar_wait(s_full, nv & 1, a.ctx, abort_flag))) break;
+        tc_fence_after();
+        const float* nl = vec + st * 2 * kT;
+        const float* dd = nl + kT;
+        float p[kT];
+        tmem_ld32f(lb + C::S_COL, p);
+        tmem_ld32f(lb + C::S_COL + 32, p + 32);
+        tmem_ld32f(lb + C::S_COL + 64, p + 64);
+        tmem_ld32f(lb + C::S_COL + 96, p + 96);
+        tmem_ld_wait();
+        reg_fence32(p);
+        reg_fence32(p + 32);
+        reg_fence32(p + 64);
+        reg_fence32(p + 96);
+        // p = 2^(s scale log2(e) - LSE log2(e)); padding rows carry -inf
+#pragma unroll
+        for (int c = 0; c < kT; c += 2) {
+          const float2 n2 = *reinterpret_cast<const float2*>(nl + c);
+          const float2 x = __ffma2_rn(make_float2(p[c], p[c + 1]), sc2, n2);
+          p[c] = fast_exp2(x.x);
+          p[c + 1] = fast_exp2(x.y);
+        }
+        if (w.cls == kPartial || it.klen < kT) {
+          // key `row` is visible to query column q iff q >= qmin
+          long long qmin = 0;
+          if (a.causal)
+            qmin = row + it.k0 - w.q0 - floor_div(w.qoff - it.koff, a.stride);
+          if (row >= it.klen) qmin = kT;
+          const int qm = qmin < 0 ? 0 : (qmin > kT ? kT : static_cast<int>(qmin));
+#pragma unroll
+          for (int c = 0; c < kT; ++c)
+            if (c < qm) p[c] = 0.f;
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < kT; c0 += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) pk[c >> 1] = pack_bf16x2(p[c0 + c], p[c0 + c + 1]);
+          tmem_st16(lb + C::S_COL + (c0 >> 1), pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        if (!(ok = mbar_wait(dp_full, nv & 1, a.ctx, abort_flag))) break;
+        tc_fence_after();
+        // dS^T = P^T (dP^T - D) -> bf16 rows of 64 queries, 128-byte swizzle
+#pragma unroll
+        for (int c0 = 0; c0 < kT; c0 += 64) {
+          float dp[64];
+          tmem_ld32f(lb + C::DP_COL + c0, dp);
+          tmem_ld32f(lb + C::DP_COL + c0 + 32, dp + 32);
+          tmem_ld_wait();
+          reg_fence32(dp);
+          reg_fence32(dp + 32);
+          uint8_t* atom = ds_row + (c0 / 64) * kBox;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = g * 8 + e * 2;
+              const float2 d2 = *reinterpret_cast<const float2*>(dd + c0 + c);
+              w4[e] = pack_bf16x2(p[c0 + c] * (dp[c] - d2.x), p[c0 + c + 1] * (dp[c + 1] - d2.y));
+            }
+            *reinterpret_cast<uint4*>(atom + ((g ^ sw) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(ds_full);
+        ++nv;
+        ++nq;
+      }
+    }
+  } else if (warp >= 8) {
+    // ----------------------------------------- reduce: dQ out, dK / dV out --
+    regs_dec<kRegsReduce>();
+    const int row = threadIdx.x & 127;
+    const uint32_t lb = tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
+    uint32_t nv = 0, nacc = 0;
+    BItem it;
+    bool ok = true;
+    for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
+      QWalk w;
+      w.start(a, it);
+      int qt, h;
+      bool any = false;
+      while (w.next(a, it, qt, h)) {
+        if (!(ok = mbar_wait(dq_full, nv & 1, a.ctx, abort_flag))) break;
+        tc_fence_after();
+        float acc[DQK];
+#pragma unroll
+        for (int c0 = 0; c0 < DQK; c0 += 32) tmem_ld32f(lb + C::DQ_COL + c0, acc + c0);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c0 = 0; c0 < DQK; c0 += 32) reg_fence32(acc + c0);
+        tc_fence_before();
+        mbar_arrive(dq_empty);
+        const int bh = it.b * a.Hq + h;
+        float* dst = a.ws_dq + (static_cast<long long>(bh) * a.ntq_ws + qt) * DQK * kT + row;
+#pragma unroll
+        for (int c = 0; c < DQK; ++c) atomicAdd(dst + c * kT, acc[c]);
+        ++nv;
+        any = true;
+      }
+      if (!ok) break;
+      if (any) {
+        if (!(ok = mbar_wait(acc_full, nacc & 1, a.ctx, abort_flag))) break;
+        tc_fence_after();
+      }
+      const bool valid = row < it.klen;
+      const long long krow = static_cast<long long>(it.bkv) * a.n_k + it.k0 + row;
+      store_key_grad<DV>(lb + C::DV_COL, any, valid, 1.f, a.dv, krow, a.block_mode);
+      store_key_grad<DQK>(lb + C::DK_COL, any, valid, a.scale, a.dk, krow, a.block_mode);
+      if (any) {
+        tc_fence_before();
+        mbar_arrive(acc_empty);
+        ++nacc;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------- teardown --
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_flag && threadIdx.x == 0) {
+    // let in-flight loads land before shared memory is released (bounded)
+    const int nk = *kv_issued;
+    if (nk > 0) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(kv_full, (nk - 1) & 1) && globaltimer_ns() - t0 < a.ctx.wait_ns) {
+      }
+    }
+    const int nq = *q_issued;
+    for (int i = nq - 2 < 0 ? 0 : nq - 2; i < nq; ++i) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(&q_full[i & 1], (i >> 1) & 1) &&
+             globaltimer_ns() - t0 < a.ctx.wait_ns) {
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------- prep / out --
+
+struct PrepArgs {
+  const void* out;     // forward output (D = rowsum(dO * O)), or null
+  const void* dout;
+  const float* delta;  // caller's D, used when out is null
+  const float* lse;    // forward LSE, or null (delta-only mode)
+  int n_q, d_v;
+  int row_pitch;       // rows per head in the destination arrays
+  long long rows;      // B * Hq * row_pitch
+  float* nl2;          // [rows] or null
+  float* d_ws;         // [rows] or null
+  float* dq_ws;        // zeroed when non-null
+  long long dq_floats;
+  float* delta_out;    // [B * Hq * n_q] or null
+};
+
+// One warp per destination row.
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(PrepArgs p) {
+  const int wpb = blockDim.x >> 5;
+  const long long nw = static_cast<long long>(gridDim.x) * wpb;
+  const long long gw = static_cast<long long>(blockIdx.x) * wpb + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (long long r = gw; r < p.rows; r += nw) {
+    const long long bh = r / p.row_pitch;
+    const int t = static_cast<int>(r % p.row_pitch);
+    float dsum = 0.f, nl = -INFINITY;
+    if (t < p.n_q) {
+      const long long src = bh * p.n_q + t;
+      if (p.out != nullptr) {
+        const T* o = static_cast<const T*>(p.out) + src * p.d_v;
+        const T* g = static_cast<const T*>(p.dout) + src * p.d_v;
+        for (int c = lane; c < p.d_v; c += 32) dsum += to_f32(o[c]) * to_f32(g[c]);
+#pragma unroll
+        for (int s = 16; s > 0; s >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, s);
+      } else {
+        dsum = p.delta[src];
+      }
+      if (p.lse != nullptr) {
+        const float l = p.lse[src];
+        nl = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
+      }
+    }
+    if (lane == 0) {
+      if (p.d_ws) p.d_ws[r] = dsum;
+      if (p.nl2) p.nl2[r] = nl;
+      if (p.delta_out && t < p.n_q) p.delta_out[bh * p.n_q + t] = dsum;
+    }
+  }
+  if (p.dq_ws != nullptr) {
+    float4* z = reinterpret_cast<float4*>(p.dq_ws);
+    const long long n4 = p.dq_floats / 4;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+      z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// dQ = scale * workspace (ring: stored in the output dtype) or dQ += scale *
+// workspace (block: fp32 accumulator).  One CTA per (head, 128-row tile); 32
+// columns at a time pass through shared memory to turn the workspace's
+// column-major tile into row-major rows.
+template <typename T, bool ACCUM>
+__global__ void __launch_bounds__(256) bwd_dq_finalize_kernel(const float* ws, T* dq, float scale,
+                                                              int n_q, int d_qk, int ntq) {
+  __shared__ float tile[32][kT + 1];
+  const long long bh = blockIdx.x / ntq;
+  const int qt = blockIdx.x % ntq;
+  const float* src = ws + (bh * ntq + qt) * static_cast<long long>(d_qk) * kT;
+  const int t0 = qt * kT;
+  for (int c0 = 0; c0 < d_qk; c0 += 32) {
+    for (int i = threadIdx.x; i < 32 * kT; i += blockDim.x)
+      tile[i / kT][i % kT] = src[static_cast<long long>(c0) * kT + i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * kT; i += blockDim.x) {
+      const int r = i / 32, c = i % 32;
+      if (t0 + r < n_q) {
+        T* d = dq + (bh * n_q + t0 + r) * d_qk + c0 + c;
+        const float x = tile[c][r] * scale;
+        if constexpr (ACCUM) {
+          *d = *d + x;
+        } else {
+          *d = from_f32<T>(x);
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <int DQK, int DV>
+int launch_bwd_typed(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& tdo, const BwdArgs& args, int grid, cudaStream_t stream) {
+  auto kern = bwd_tc_kernel<DQK, DV>;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return RA_ERR_CUDA;
+  if (fa.numRegs > kRegsLaunch) return RA_ERR_UNSUPPORTED;  // the register split would not fit
+  constexpr int smem = BCfg<DQK, DV>::SMEM;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return RA_ERR_CUDA;
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, args);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+int launch_prep(const PrepArgs& p, ra_dtype dt, const DeviceInfo& dev, cudaStream_t st) {
+  const long long blocks_rows = (p.rows + 7) / 8;
+  long long blocks = blocks_rows < 4LL * dev.num_sms ? blocks_rows : 4LL * dev.num_sms;
+  if (blocks < 1) blocks = 1;
+  if (dt == RA_BF16)
+    bwd_prep_kernel<__nv_bfloat16><<<static_cast<int>(blocks), 256, 0, st>>>(p);
+  else
+    bwd_prep_kernel<float><<<static_cast<int>(blocks), 256, 0, st>>>(p);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(const ra_shape& s) {
+  return bwd_layout(s.B, s.Hq, s.n_q, s.d_qk).total;
+}
+
+int launch_backward_delta(const void* out, const void* dout, const ra_shape& s, float* delta,
+                          const DeviceInfo& dev, cudaStream_t stream) {
+  PrepArgs p{};
+  p.out = out;
+  p.dout = dout;
+  p.n_q = s.n_q;
+  p.d_v = s.d_v;
+  p.row_pitch = s.n_q;
+  p.rows = static_cast<long long>(s.B) * s.Hq * s.n_q;
+  p.delta_out = delta;
+  return launch_prep(p, s.dtype, dev, stream);
+}
+
+int launch_backward(const void* q, const void* k, const void* v, const void* out,
+                    const float* lse, const void* dout, const float* delta, const ra_shape& s,
+                    int P, int q_offset, int k_offset, long long stride, int causal, int striped,
+                    float scale, void* dq, void* dk, void* dv, bool block_mode, void* workspace,
+                    const DeviceInfo& dev, cudaStream_t stream) {
+  const BwdLayout L = bwd_layout(s.B, s.Hq, s.n_q, s.d_qk);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* ws_dq = reinterpret_cast<float*>(ws + L.dq_off);
+  float* ws_nl2 = reinterpret_cast<float*>(ws + L.nl2_off);
+  float* ws_d = reinterpret_cast<float*>(ws + L.d_off);
+
+  PrepArgs p{};
+  p.out = block_mode ? nullptr : out;
+  p.dout = dout;
+  p.delta = delta;
+  p.lse = lse;
+  p.n_q = s.n_q;
+  p.d_v = s.d_v;
+  p.row_pitch = L.ntq * kBwdTile;
+  p.rows = L.rows_pad;
+  p.nl2 = ws_nl2;
+  p.d_ws = ws_d;
+  p.dq_ws = ws_dq;
+  p.dq_floats = L.rows_pad * s.d_qk;
+  int rc = launch_prep(p, s.dtype, dev, stream);
+  if (rc != RA_OK) return rc;
+
+  BwdArgs a{};
+  a.B = s.B;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.n_q = s.n_q;
+  a.n_k = s.n_k;
+  a.P = P;
+  a.grp = s.Hq / s.Hkv;
+  a.q_offset = q_offset;
+  a.k_offset = k_offset;
+  a.causal = causal;
+  a.striped = striped;
+  a.stride = striped ? P : stride;
+  a.scale = scale;
+  a.scale_log2 = scale * kLog2e;
+  a.ntq_ws = L.ntq;
+  a.ws_dq = ws_dq;
+  a.ws_nl2 = ws_nl2;
+  a.ws_d = ws_d;
+  a.dk = dk;
+  a.dv = dv;
+  a.block_mode = block_mode ? 1 : 0;
+  a.ctx = dev.ctx;
+
+  if (s.dtype == RA_BF16) {
+    a.tq = a.tk = kT;
+    a.ntq = L.ntq;
+    a.ntk = (s.n_k + kT - 1) / kT;
+    const long long items = static_cast<long long>(s.B) * s.Hkv * a.ntk;
+    if (items > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+    a.items = static_cast<int>(items);
+    CUtensorMap tq, tk, tv, tdo;
+    const uint64_t hq = static_cast<uint64_t>(s.B) * s.Hq;
+    const uint64_t hkv = static_cast<uint64_t>(s.B) * s.Hkv;
+    if (make_tmap_bf16_3d(&tq, q, s.d_qk, s.n_q, hq, s.d_qk * 2ull,
+                          static_cast<uint64_t>(s.n_q) * s.d_qk * 2, 64, kT) != 0 ||
+        make_tmap_bf16_3d(&tk, k, s.d_qk, s.n_k, hkv, s.d_qk * 2ull,
+                          static_cast<uint64_t>(s.n_k) * s.d_qk * 2, 64, kT) != 0 ||
+        make_tmap_bf16_3d(&tv, v, s.d_v, s.n_k, hkv, s.d_v * 2ull,
+                          static_cast<uint64_t>(s.n_k) * s.d_v * 2, 64, kT) != 0 ||
+        make_tmap_bf16_3d(&tdo, dout, s.d_v, s.n_q, hq, s.d_v * 2ull,
+                          static_cast<uint64_t>(s.n_q) * s.d_v * 2, 64, kT) != 0)
+      return RA_ERR_CUDA;
+    const int grid = a.items < dev.num_sms ? a.items : dev.num_sms;
+    if (s.d_qk == 128 && s.d_v == 128) rc = launch_bwd_typed<128, 128>(tq, tk, tv, tdo, a, grid, stream);
+    else if (s.d_qk == 64 && s.d_v == 64) rc = launch_bwd_typed<64, 64>(tq, tk, tv, tdo, a, grid, stream);
+    else if (s.d_qk == 64 && s.d_v == 128) rc = launch_bwd_typed<64, 128>(tq, tk, tv, tdo, a, grid, stream);
+    else if (s.d_qk == 128 && s.d_v == 64) rc = launch_bwd_typed<128, 64>(tq, tk, tv, tdo, a, grid, stream);
+    else return RA_ERR_UNSUPPORTED;
+  } else {
+    rc = launch_simt_backward(q, k, v, dout, s, a, dev, stream);
+  }
+  if (rc != RA_OK) return rc;
+
+  const long long blocks = static_cast<long long>(s.B) * s.Hq * L.ntq;
+  if (blocks > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  if (block_mode) {
+    bwd_dq_finalize_kernel<float, true><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        ws_dq, static_cast<float*>(dq), scale, s.n_q, s.d_qk, L.ntq);
+  } else if (s.dtype == RA_BF16) {
+    bwd_dq_finalize_kernel<__nv_bfloat16, false><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        ws_dq, static_cast<__nv_bfloat16*>(dq), scale, s.n_q, s.d_qk, L.ntq);
+  } else {
+    bwd_dq_finalize_kernel<float, false><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        ws_dq, static_cast<float*>(dq), scale, s.n_q, s.d_qk, L.ntq);
+  }
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+}  // namespace ra

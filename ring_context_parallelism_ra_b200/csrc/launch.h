@@ -55,6 +55,23 @@ int launch_decode_partial_static(const void* q, const void* k, const void* v,
                                  float* o_part, float* lse_part, const DeviceInfo& dev,
                                  cudaStream_t stream);
 
+// Backward pass (bwd_attention.cu, bwd_simt.cu).  Ring mode (block_mode
+// false): dq, dk, dv are outputs of the input dtype and D is computed from
+// out / dout.  Block mode: dq, dk, dv are fp32 accumulators (+=) and D comes
+// from `delta`.  `workspace` holds at least backward_workspace_bytes(s).
+size_t backward_workspace_bytes(const ra_shape& s);
+int launch_backward(const void* q, const void* k, const void* v, const void* out,
+                    const float* lse, const void* dout, const float* delta, const ra_shape& s,
+                    int P, int q_offset, int k_offset, long long stride, int causal, int striped,
+                    float scale, void* dq, void* dk, void* dv, bool block_mode, void* workspace,
+                    const DeviceInfo& dev, cudaStream_t stream);
+int launch_backward_delta(const void* out, const void* dout, const ra_shape& s, float* delta,
+                          const DeviceInfo& dev, cudaStream_t stream);
+struct BwdArgs;
+int launch_simt_backward(const void* q, const void* k, const void* v, const void* dout,
+                         const ra_shape& s, BwdArgs a, const DeviceInfo& dev,
+                         cudaStream_t stream);
+
 int launch_block_class(int n_q, int n_k, int q_block, int k_block, int q_offset, int k_offset,
                        int causal, int8_t* map_dev, cudaStream_t stream);
 

@@ -85,6 +85,32 @@ int check_ring_args(const void* q, const void* k, const void* v, int P, int caus
   return check_attention_dims(shape);
 }
 
+int check_backward_dims(const ra_shape* s) {
+  if ((s->d_qk == 64 || s->d_qk == 128) && (s->d_v == 64 || s->d_v == 128)) return RA_OK;
+  return RA_ERR_UNSUPPORTED;
+}
+
+int check_ring_backward_args(const void* q, const void* k, const void* v, const void* out,
+                             const float* lse, const void* dout, int P, int causal,
+                             const void* dq, const void* dk, const void* dv,
+                             const ra_shape* shape, const void* workspace,
+                             size_t workspace_bytes) {
+  int rc = check_common(shape);
+  if (rc != RA_OK) return rc;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace))
+    return RA_ERR_INVALID;
+  if (P < 1 || shape->n_q != shape->n_k || shape->n_q % P != 0) return RA_ERR_INVALID;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID;
+  rc = check_backward_dims(shape);
+  if (rc != RA_OK) return rc;
+  if (workspace_bytes < backward_workspace_bytes(*shape)) return RA_ERR_INVALID;
+  return RA_OK;
+}
+
 __global__ void block_class_kernel(int n_q, int n_k, int q_block, int k_block, int q_offset,
                                    int k_offset, int causal, int tq, int tk, int8_t* map) {
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -299,6 +325,78 @@ int ra_block_class_device(int n_q, int n_k, int q_block, int k_block, int q_offs
     return RA_ERR_INVALID;
   return launch_block_class(n_q, n_k, q_block, k_block, q_offset, k_offset, causal, map_dev,
                             static_cast<cudaStream_t>(stream));
+}
+
+size_t ra_backward_workspace_bytes(const ra_shape* shape) {
+  if (check_common(shape) != RA_OK) return 0;
+  return backward_workspace_bytes(*shape);
+}
+
+int ra_backward_delta(const void* out, const void* dout, const ra_shape* shape, float* delta,
+                      void* stream) {
+  int rc = check_common(shape);
+  if (rc != RA_OK) return rc;
+  if (!out || !dout || !delta) return RA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(delta)) return RA_ERR_INVALID;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc != RA_OK) return rc;
+  return launch_backward_delta(out, dout, *shape, delta, dev, static_cast<cudaStream_t>(stream));
+}
+
+int ra_ring_backward(const void* q, const void* k, const void* v, const void* out,
+                     const float* lse, const void* dout, int P, int causal, float scale, void* dq,
+                     void* dk, void* dv, const ra_shape* shape, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  int rc = check_ring_backward_args(q, k, v, out, lse, dout, P, causal, dq, dk, dv, shape,
+                                    workspace, workspace_bytes);
+  if (rc != RA_OK) return rc;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc != RA_OK) return rc;
+  return launch_backward(q, k, v, out, lse, dout, nullptr, *shape, P, 0, 0, 1, causal, 0, scale,
+                         dq, dk, dv, false, workspace, dev, static_cast<cudaStream_t>(stream));
+}
+
+int ra_ring_backward_striped(const void* q, const void* k, const void* v, const void* out,
+                             const float* lse, const void* dout, int P, int causal, float scale,
+                             void* dq, void* dk, void* dv, const ra_shape* shape, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  int rc = check_ring_backward_args(q, k, v, out, lse, dout, P, causal, dq, dk, dv, shape,
+                                    workspace, workspace_bytes);
+  if (rc != RA_OK) return rc;
+  if ((shape->n_q / P) % 128 != 0) return RA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc != RA_OK) return rc;
+  return launch_backward(q, k, v, out, lse, dout, nullptr, *shape, P, 0, 0, P, causal, 1, scale,
+                         dq, dk, dv, false, workspace, dev, static_cast<cudaStream_t>(stream));
+}
+
+int ra_block_backward(const void* q, const void* k, const void* v, const void* dout,
+                      const float* lse, const float* delta, const ra_shape* shape, int q_offset,
+                      int k_offset, int pos_stride, int causal, float scale, float* dq_acc,
+                      float* dk_acc, float* dv_acc, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  int rc = check_common(shape);
+  if (rc != RA_OK) return rc;
+  if (!q || !k || !v || !dout || !lse || !delta || !dq_acc || !dk_acc || !dv_acc || !workspace)
+    return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(delta) || !aligned16(dq_acc) || !aligned16(dk_acc) || !aligned16(dv_acc) ||
+      !aligned16(workspace))
+    return RA_ERR_INVALID;
+  if ((causal != 0 && causal != 1) || q_offset < 0 || k_offset < 0 || pos_stride < 1)
+    return RA_ERR_INVALID;
+  rc = check_backward_dims(shape);
+  if (rc != RA_OK) return rc;
+  if (workspace_bytes < backward_workspace_bytes(*shape)) return RA_ERR_INVALID;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc != RA_OK) return rc;
+  return launch_backward(q, k, v, nullptr, lse, dout, delta, *shape, 1, q_offset, k_offset,
+                         pos_stride, causal, 0, scale, dq_acc, dk_acc, dv_acc, true, workspace,
+                         dev, static_cast<cudaStream_t>(stream));
 }
 
 int ra_get_status(void* stream) {

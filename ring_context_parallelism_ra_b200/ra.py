@@ -21,7 +21,9 @@ __all__ = [
     "lse_merge", "ring_forward", "ring_forward_striped",
     "ring_forward_host", "decode_workspace_bytes", "decode_partial", "decode_partial_noalloc",
     "decode_merge",
-    "decode_pass_q", "block_class", "block_class_device", "get_status", "set_wait_limit_ns",
+    "decode_pass_q", "backward_workspace_bytes", "backward_delta", "ring_backward",
+    "ring_backward_striped", "block_backward",
+    "block_class", "block_class_device", "get_status", "set_wait_limit_ns",
     "check_wait_timeout", "launch_count", "status_string", "EXPORTED",
 ]
 
@@ -32,7 +34,9 @@ RA_F32, RA_BF16 = 0, 1
 EXPORTED = (
     "ra_block_partial", "ra_block_partial_strided", "ra_lse_merge", "ra_ring_forward",
     "ra_ring_forward_striped", "ra_decode_workspace_bytes",
-    "ra_decode_partial", "ra_decode_partial_noalloc", "ra_decode_merge", "ra_block_class", "ra_block_class_device",
+    "ra_decode_partial", "ra_decode_partial_noalloc", "ra_decode_merge",
+    "ra_backward_workspace_bytes", "ra_backward_delta", "ra_ring_backward",
+    "ra_ring_backward_striped", "ra_block_backward", "ra_block_class", "ra_block_class_device",
     "ra_get_status", "ra_set_wait_limit_ns", "ra_check_wait_timeout", "ra_status_string",
     "ra_launch_count", "ra_shutdown",
 )
@@ -82,6 +86,13 @@ def lib() -> ctypes.CDLL:
             "ra_decode_partial": (i, [vp, vp, vp, ctypes.c_longlong, sp, f, vp, vp, vp, sz, vp]),
             "ra_decode_partial_noalloc": (i, [vp, vp, vp, ctypes.c_longlong, sp, f, vp, vp, vp]),
             "ra_decode_merge": (i, [vp, vp, i, sp, vp, i, vp, vp]),
+            "ra_backward_workspace_bytes": (sz, [sp]),
+            "ra_backward_delta": (i, [vp, vp, sp, vp, vp]),
+            "ra_ring_backward": (i, [vp, vp, vp, vp, vp, vp, i, i, f, vp, vp, vp, sp, vp, sz, vp]),
+            "ra_ring_backward_striped": (i, [vp, vp, vp, vp, vp, vp, i, i, f, vp, vp, vp, sp, vp,
+                                             sz, vp]),
+            "ra_block_backward": (i, [vp, vp, vp, vp, vp, vp, sp, i, i, i, i, f, vp, vp, vp, vp,
+                                      sz, vp]),
             "ra_block_class": (i, [i, i, i, i, i, i, i, vp]),
             "ra_block_class_device": (i, [i, i, i, i, i, i, i, vp, vp]),
             "ra_get_status": (i, [vp]),
@@ -245,6 +256,86 @@ def ring_forward_host(q, k, v, P, causal=True, scale=None, device="cuda", bufs=N
     lse_h.copy_(lse, non_blocking=True)
     torch.cuda.current_stream().synchronize()
     return out_h, lse_h
+
+
+def backward_workspace_bytes(q, k, v) -> int:
+    s = _shape(q, k, v)
+    return int(lib().ra_backward_workspace_bytes(ctypes.byref(s)))
+
+
+def _workspace(q, k, v, workspace):
+    need = backward_workspace_bytes(q, k, v)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    return ctypes.c_void_p(workspace.data_ptr()), ctypes.c_size_t(
+        workspace.numel() * workspace.element_size())
+
+
+def backward_delta(out, dout, delta=None, stream=None):
+    """D = rowsum(dO * O) per query row: fp32 [B, Hq, n_q]."""
+    B, Hq, n, dv = out.shape
+    if dout.shape != out.shape:
+        raise ValueError("dout must be shaped like out")
+    if delta is None:
+        delta = torch.empty((B, Hq, n), device=out.device, dtype=torch.float32)
+    s = Shape(B, Hq, Hq, n, n, dv, dv, _dtype_code(out.dtype))
+    rc = lib().ra_backward_delta(_need(out, "out"), _need(dout, "dout", out.dtype), ctypes.byref(s),
+                                 _need(delta, "delta", torch.float32), _stream(stream))
+    _check("ra_backward_delta", rc)
+    return delta
+
+
+def _ring_backward(name, q, k, v, out, lse, dout, P, causal, scale, dq, dk, dv, workspace,
+                   stream):
+    s = _shape(q, k, v)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    wp, wb = _workspace(q, k, v, workspace)
+    rc = getattr(lib(), name)(
+        _need(q, "q"), _need(k, "k", q.dtype), _need(v, "v", q.dtype), _need(out, "out", q.dtype),
+        _need(lse, "lse", torch.float32), _need(dout, "dout", q.dtype), int(P), int(bool(causal)),
+        float(scale), _need(dq, "dq", q.dtype), _need(dk, "dk", q.dtype), _need(dv, "dv", q.dtype),
+        ctypes.byref(s), wp, wb, _stream(stream))
+    _check(name, rc)
+    return dq, dk, dv
+
+
+def ring_backward(q, k, v, out, lse, dout, P, causal=True, scale=None, dq=None, dk=None,
+                  dv=None, workspace=None, stream=None):
+    """Gradients (dQ, dK, dV) of ring_forward, in the input dtype."""
+    return _ring_backward("ra_ring_backward", q, k, v, out, lse, dout, P, causal, scale, dq, dk,
+                          dv, workspace, stream)
+
+
+def ring_backward_striped(q, k, v, out, lse, dout, P, causal=True, scale=None, dq=None, dk=None,
+                          dv=None, workspace=None, stream=None):
+    """Gradients of ring_forward_striped (striped row order throughout)."""
+    return _ring_backward("ra_ring_backward_striped", q, k, v, out, lse, dout, P, causal, scale,
+                          dq, dk, dv, workspace, stream)
+
+
+def block_backward(q, k, v, dout, lse, delta, q_offset=0, k_offset=0, pos_stride=1, causal=True,
+                   scale=None, dq_acc=None, dk_acc=None, dv_acc=None, workspace=None,
+                   stream=None):
+    """Add one block's gradient shares into fp32 accumulators (zeros when not
+    given); lse / delta are the query rows' final statistics."""
+    s = _shape(q, k, v)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    f32 = torch.float32
+    dq_acc = torch.zeros(q.shape, device=q.device, dtype=f32) if dq_acc is None else dq_acc
+    dk_acc = torch.zeros(k.shape, device=q.device, dtype=f32) if dk_acc is None else dk_acc
+    dv_acc = torch.zeros(v.shape, device=q.device, dtype=f32) if dv_acc is None else dv_acc
+    wp, wb = _workspace(q, k, v, workspace)
+    rc = lib().ra_block_backward(
+        _need(q, "q"), _need(k, "k", q.dtype), _need(v, "v", q.dtype), _need(dout, "dout", q.dtype),
+        _need(lse, "lse", f32), _need(delta, "delta", f32), ctypes.byref(s), int(q_offset),
+        int(k_offset), int(pos_stride), int(bool(causal)), float(scale),
+        _need(dq_acc, "dq_acc", f32), _need(dk_acc, "dk_acc", f32), _need(dv_acc, "dv_acc", f32),
+        wp, wb, _stream(stream))
+    _check("ra_block_backward", rc)
+    return dq_acc, dk_acc, dv_acc
 
 
 def decode_workspace_bytes(B, Hq, Hkv, n_k, d=128) -> int:

@@ -25,10 +25,11 @@ from dataclasses import dataclass, field
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "workload", "draw_slice", "make_qkv",
-           "make_workload_inputs", "prefill_flops", "decode_kv_bytes", "striped_order"]
+__all__ = ["Workload", "WORKLOADS", "workload", "draw_slice", "make_qkv", "make_dout",
+           "make_workload_inputs", "prefill_flops", "backward_flops", "decode_kv_bytes",
+           "striped_order"]
 
-_TENSOR_ID = {"q": 1, "k": 2, "v": 3}
+_TENSOR_ID = {"q": 1, "k": 2, "v": 3, "do": 4}
 
 
 @dataclass(frozen=True)
@@ -92,6 +93,15 @@ def draw_slice(seed: int, tensor: str, b: int, h: int, rows: int, d: int,
     return x.to(dtype)
 
 
+def make_dout(B, Hq, n_q, d_v, dtype=torch.bfloat16, seed=0, device="cpu"):
+    """Gradient arriving at the output, dO [B, Hq, n_q, d_v]: N(0,1) rounded."""
+    g = torch.empty((B, Hq, n_q, d_v), dtype=dtype, device=device)
+    for b in range(B):
+        for h in range(Hq):
+            g[b, h] = draw_slice(seed, "do", b, h, n_q, d_v, dtype, 1.0, device)
+    return g
+
+
 def make_qkv(B, Hq, Hkv, n_q, n_k, d_qk, d_v, dtype=torch.bfloat16, seed=0,
              qk_mult=1.0, device="cpu"):
     """Contiguous BHSD tensors q [B,Hq,n_q,d_qk], k [B,Hkv,n_k,d_qk],
@@ -117,6 +127,14 @@ def make_workload_inputs(wl: Workload, device="cpu"):
 def prefill_flops(wl: Workload) -> float:
     """Algorithmic FLOPs of QK^T and PV over all heads; causal counts half."""
     f = 2.0 * wl.B * wl.Hq * wl.n * wl.n * (wl.d_qk + wl.d_v)
+    return f / 2 if wl.causal else f
+
+
+def backward_flops(wl: Workload) -> float:
+    """Algorithmic FLOPs of the backward pass over all heads: the scores
+    recomputed, dP = dO V^T, dV = P^T dO, dQ = dS K, dK = dS^T Q; causal
+    counts half."""
+    f = 2.0 * wl.B * wl.Hq * wl.n * wl.n * (3 * wl.d_qk + 2 * wl.d_v)
     return f / 2 if wl.causal else f
 
 

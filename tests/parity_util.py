@@ -3,6 +3,14 @@
 Bars (stated for the method's outputs): bf16 inputs with fp32 accumulation
 give O within max-abs 2e-2 and mean-abs 2e-3 of the fp64 definition; fp32
 inputs give O within 1e-4; the log-sum-exp within 1e-3.
+
+Gradients (backward pass) take the same bars in units of their own size
+when that exceeds 1: O is a convex combination of the values (|O| is at most
+max |v|, about 4 for N(0,1) inputs), a gradient is not.  Every rounding in
+the bf16 backward (P and dS to bf16 before their products, the forward's O
+in bf16 inside D = rowsum(dO * O), the bf16 results) is relative, so its
+error scales with the gradient: max-abs err <= 2e-2 * max(1, max |ref|) and
+mean-abs err <= 2e-3 * max(1, mean |ref|); fp32: 1e-4 * max(1, max |ref|).
 """
 import numpy as np
 import torch
@@ -44,3 +52,22 @@ def check_lse(got, want, what="LSE"):
     mx = float(np.abs(g[fin] - w[fin]).max()) if fin.any() else 0.0
     assert mx <= LSE_MAX_ABS, f"{what}: max abs {mx:.3g} > {LSE_MAX_ABS}"
     return mx
+
+
+def check_grad(got, want, dtype, what="grad"):
+    """Element-wise comparison of a gradient against the oracle, with the bars
+    scaled by the reference's magnitude when it exceeds 1."""
+    g, w = to64(got), to64(want)
+    assert g.shape == w.shape, (g.shape, w.shape)
+    assert np.isfinite(g).all(), f"{what}: non-finite values"
+    err = np.abs(g - w)
+    mx, mean = float(err.max()), float(err.mean())
+    s_max = max(1.0, float(np.abs(w).max()))
+    s_mean = max(1.0, float(np.abs(w).mean()))
+    if dtype in ("f32", torch.float32):
+        assert mx <= F32_MAX_ABS * s_max, f"{what}: max abs {mx:.3g} > {F32_MAX_ABS} x {s_max:.3g}"
+    else:
+        assert mx <= BF16_MAX_ABS * s_max, f"{what}: max abs {mx:.3g} > {BF16_MAX_ABS} x {s_max:.3g}"
+        assert mean <= BF16_MEAN_ABS * s_mean, \
+            f"{what}: mean abs {mean:.3g} > {BF16_MEAN_ABS} x {s_mean:.3g}"
+    return mx, mean

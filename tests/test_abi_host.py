@@ -102,3 +102,55 @@ def test_decode_workspace_size_is_chunk_partials():
     n = ra.decode_workspace_bytes(4, 64, 8, 131072)
     assert n >= 64 * 4 * 64 * 129 * 4
     assert n < 64 * 4 * 64 * 129 * 4 + 4096
+
+
+def test_backward_validation_rejects_bad_arguments_before_launch():
+    L = ra.lib()
+    p = ctypes.c_void_p(256)
+    nul = ctypes.c_void_p(0)
+    mis = ctypes.c_void_p(264)
+    INV, UNS = ra.RA_ERR_INVALID, ra.RA_ERR_UNSUPPORTED
+    s = _shape()
+    ws = L.ra_backward_workspace_bytes(ctypes.byref(s))
+    big = ctypes.c_size_t(ws)
+
+    def ring(fn, shape, P=1, causal=1, q=p, wsb=big):
+        return fn(q, p, p, p, p, p, P, causal, 1.0, p, p, p, ctypes.byref(shape), p, wsb, nul)
+
+    for fn in (L.ra_ring_backward, L.ra_ring_backward_striped):
+        assert ring(fn, s, q=nul) == INV
+        assert ring(fn, s, q=mis) == INV
+        assert ring(fn, s, P=0) == INV
+        assert ring(fn, s, P=3) == INV                       # 128 % 3
+        assert ring(fn, s, causal=2) == INV
+        assert ring(fn, _shape(n_k=64)) == INV               # n_q != n_k
+        assert ring(fn, _shape(d_qk=192)) == UNS             # no backward for D_qk = 192
+        assert ring(fn, _shape(dtype=ra.RA_F32, d_v=32)) == UNS
+        assert ring(fn, s, wsb=ctypes.c_size_t(ws - 1)) == INV
+    # striped needs whole 128-row tiles per partition
+    s_odd = _shape(n_q=384, n_k=384)
+    ws_odd = ctypes.c_size_t(L.ra_backward_workspace_bytes(ctypes.byref(s_odd)))
+    assert ring(L.ra_ring_backward_striped, s_odd, P=2, wsb=ws_odd) == UNS   # 192-row partitions
+
+    def blk(shape, qo=0, ko=0, st=1, causal=1, lse=p, wsb=big):
+        return L.ra_block_backward(p, p, p, p, lse, p, ctypes.byref(shape), qo, ko, st, causal,
+                                   1.0, p, p, p, p, wsb, nul)
+
+    assert blk(s, lse=nul) == INV
+    assert blk(s, qo=-1) == INV
+    assert blk(s, st=0) == INV
+    assert blk(s, causal=3) == INV
+    assert blk(_shape(Hq=3, Hkv=2)) == INV
+    assert blk(_shape(d_qk=192)) == UNS
+    assert blk(s, wsb=ctypes.c_size_t(0)) == INV
+    assert L.ra_backward_delta(nul, p, ctypes.byref(s), p, nul) == INV
+    assert L.ra_backward_delta(p, p, None, p, nul) == INV
+
+
+def test_backward_workspace_size():
+    # fp32 dQ accumulator plus two row vectors, rows padded to 128 per head
+    for B, H, n, d in [(1, 8, 8192, 128), (2, 3, 1000, 64)]:
+        s = _shape(B=B, Hq=H, Hkv=1, n_q=n, n_k=n, d_qk=d, d_v=d)
+        rows = B * H * ((n + 127) // 128) * 128
+        got = ra.lib().ra_backward_workspace_bytes(ctypes.byref(s))
+        assert rows * (d + 2) * 4 <= got < rows * (d + 2) * 4 + 1024

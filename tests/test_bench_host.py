@@ -87,11 +87,15 @@ def test_reference_arm_line():
 
 
 def test_flop_and_byte_counts_match_oracle_formulas():
+    from oracle.costs import backward_flops as oracle_bwd_flops
     from oracle.costs import kv_cache_bytes, prefill_flops as oracle_flops
-    from ring_context_parallelism_ra_b200.workloads import decode_kv_bytes, prefill_flops
+    from ring_context_parallelism_ra_b200.workloads import (backward_flops, decode_kv_bytes,
+                                                           prefill_flops)
     for key in (1, 2, 3, 5):
         wl = workload(key)
         assert prefill_flops(wl) == oracle_flops(wl.B, wl.n, wl.d_qk, wl.d_v, wl.Hq, wl.causal)
+        assert backward_flops(wl) == oracle_bwd_flops(wl.B, wl.n, wl.d_qk, wl.d_v, wl.Hq,
+                                                      wl.causal)
     wl = workload(4)
     assert decode_kv_bytes(wl) == wl.B * kv_cache_bytes(1, wl.Hkv, wl.d_qk, wl.n, 2)
     assert decode_kv_bytes(wl) == 17179869184

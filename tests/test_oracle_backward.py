@@ -16,7 +16,8 @@ import pytest
 import torch
 
 from oracle.attention import attention
-from oracle.backward import attention_backward, ring_attention_backward, row_delta
+from oracle.backward import (attention_backward, attention_backward_sampled,
+                             ring_attention_backward, row_delta)
 from oracle.blockwise import striped_positions
 from oracle.costs import backward_flops, prefill_flops
 
@@ -193,3 +194,15 @@ def test_backward_flops_closed_form():
     assert backward_flops(1, 8192, 128, 128, heads=8, causal=True) == \
         5 * prefill_flops(1, 8192, 128, 128, heads=8, causal=True) // 2
     assert backward_flops(2, 100, 64, 32, heads=3) == 2 * 2 * 100 * 100 * (3 * 64 + 2 * 32) * 3
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_gradients_equal_whole_backward(causal):
+    q, k, v, g = _inputs(40, B=2, hq=4, hkv=2, nq=37, nk=37, d=6, dv=5)
+    dq, dk, dv = attention_backward(q, k, v, g, 0.4, causal)
+    rows, keys = [0, 5, 36, 17], [36, 0, 9]
+    sq, sk, sv = attention_backward_sampled(q, k, v, g, 0.4, causal, rows, keys,
+                                            heads=[3, 0], kv_heads=[1])
+    assert np.abs(sq - dq[:, [3, 0]][:, :, rows]).max() <= 1e-12
+    assert np.abs(sk - dk[:, [1]][:, :, keys]).max() <= 1e-12
+    assert np.abs(sv - dv[:, [1]][:, :, keys]).max() <= 1e-12
