@@ -28,10 +28,14 @@
 // the MN-major layout of dS.
 //
 // Tensor memory (512 columns): S^T [0,128) (P^T packed over its first 64
-// columns), dP^T [128,256), dV [256,256+DV), dK [256+DV,256+DV+DQK), dQ in its
-// own columns after dK when they fit (DQK = DV = 64, or DQK = 64, DV = 128),
-// else over the S^T columns once dV has read P^T (MMAs of one thread execute
-// in issue order; the next S^T waits until dQ has been read out).
+// columns), dP^T [128,256) (dQ over it once the compute warps have loaded
+// dP^T), dV [256,256+DV), dK [256+DV,256+DV+DQK).
+// MMA issue order per visit v: dV(v), S^T(v+1), dK(v), dQ(v), dP^T(v+1).
+// MMAs of one thread execute in issue order, so S^T(v+1) overwrites P^T(v)
+// only after dV(v) has read it, and the compute warps form P^T(v+1) while the
+// tensor cores run dK(v) and dQ(v).  A commit fires when every MMA issued
+// before it has completed: dP^T(v+1)'s also tells the compute warps that
+// dK(v) and dQ(v) are done with the dS tile.
 #include <cuda.h>
 
 #include "block_class.cuh"
@@ -79,9 +83,8 @@ struct BCfg {
   static constexpr int DP_COL = 128;
   static constexpr int DV_COL = 256;
   static constexpr int DK_COL = 256 + DV;
-  static constexpr bool DQ_OWN = 256 + DV + 2 * DQK <= 512;
-  static constexpr int DQ_COL = DQ_OWN ? 256 + DV + DQK : S_COL;
-  static_assert(DQ_OWN || DQK <= 128, "dQ must fit over the S^T columns");
+  static constexpr int DQ_COL = DP_COL;  // dQ over dP^T once dP^T has been loaded
+  static_assert(DQK <= 128 && DV <= 128, "column budget");
   static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t ID_DV = idesc_bf16_f32(128, DV, 0, 1);
   static constexpr uint32_t ID_DK = idesc_bf16_f32(128, DQK, 0, 1);
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      uint32_t nkv = 0, nq = 0, nv = 0, nacc = 0;
+      uint32_t nkv = 0, nv = 0, nacc = 0;  // nv: visits so far = query-stage counter
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ);
       const uint32_t adO = smem_u32(sdO), adS = smem_u32(sdS);
       BItem it;
@@ -313,28 +316,29 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
         QWalk w;
         w.start(a, it);
         int qt, h;
-        bool has = w.next(a, it, qt, h);
-        if (!has) continue;
+        if (!w.next(a, it, qt, h)) continue;
         if (!(ok = mbar_wait(kv_full, nkv & 1, a.ctx, abort_flag))) break;
         ++nkv;
         tc_fence_after();
-        bool first = true;
+        {  // S^T and dP^T of the item's first visit
+          const uint32_t st = nv & 1;
+          if (!(ok = mbar_wait(&q_full[st], (nv >> 1) & 1, a.ctx, abort_flag))) break;
+          tc_fence_after();
+          mma_kk<DQK>(tmem + C::S_COL, aK, aQ + st * C::QB * kBox, C::ID_S);
+          umma_commit(s_full);
+          // dP^T goes over the previous visit's dQ: wait until it is read out
+          if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
+          tc_fence_after();
+          mma_kk<DV>(tmem + C::DP_COL, aV, adO + st * C::VB * kBox, C::ID_S);
+          umma_commit(dp_full);
+        }
+        bool first = true, has = true;
         while (has) {
           int nqt, nh;
           const bool has_next = w.next(a, it, nqt, nh);
-          const int st = nq & 1;
-          if (!(ok = mbar_wait(&q_full[st], (nq >> 1) & 1, a.ctx, abort_flag))) break;
-          tc_fence_after();
+          const uint32_t st = nv & 1, st1 = (nv + 1) & 1;
           const uint32_t q_s = aQ + st * C::QB * kBox;
           const uint32_t do_s = adO + st * C::VB * kBox;
-          if (!C::DQ_OWN) {  // S^T overwrites the previous dQ: wait until it is read out
-            if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
-            tc_fence_after();
-          }
-          mma_kk<DQK>(tmem + C::S_COL, aK, q_s, C::ID_S);
-          umma_commit(s_full);
-          mma_kk<DV>(tmem + C::DP_COL, aV, do_s, C::ID_S);
-          umma_commit(dp_full);
           if (!(ok = mbar_wait(p_full, nv & 1, a.ctx, abort_flag))) break;
           tc_fence_after();
           if (first) {  // the previous item's dK, dV have been read out
@@ -342,23 +346,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
             tc_fence_after();
           }
           mma_tm(tmem + C::DV_COL, tmem + C::S_COL, do_s, C::ID_DV, !first);
+          if (has_next) {  // next S^T over P^T, which dV (issued before) has read
+            if (!(ok = mbar_wait(&q_full[st1], ((nv + 1) >> 1) & 1, a.ctx, abort_flag))) break;
+            tc_fence_after();
+            mma_kk<DQK>(tmem + C::S_COL, aK, aQ + st1 * C::QB * kBox, C::ID_S);
+            umma_commit(s_full);
+          }
           if (!(ok = mbar_wait(ds_full, nv & 1, a.ctx, abort_flag))) break;
           tc_fence_after();
           mma_km(tmem + C::DK_COL, adS, q_s, C::ID_DK, !first);
-          if (C::DQ_OWN) {
-            if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
-            tc_fence_after();
-          }
-          mma_mm(tmem + C::DQ_COL, adS, aK, C::ID_DQ);
+          mma_mm(tmem + C::DQ_COL, adS, aK, C::ID_DQ);  // dP^T was loaded before ds_full
           umma_commit(dq_full);
           umma_commit(&q_empty[st]);
-          ++nq;
-          ++nv;
-          first = false;
           if (!has_next) {
             umma_commit(acc_full);
             umma_commit(kv_empty);
             ++nacc;
+          }
+          ++nv;
+          first = false;
+          if (has_next) {  // next dP^T over this dQ, once it is read out
+            if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
+            tc_fence_after();
+            mma_kk<DV>(tmem + C::DP_COL, aV, adO + st1 * C::VB * kBox, C::ID_S);
+            umma_commit(dp_full);
           }
           qt = nqt;
           h = nh;
