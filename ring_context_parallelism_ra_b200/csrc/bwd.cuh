@@ -27,8 +27,8 @@ namespace ra {
 constexpr int kBwdTile = 128;  // rows of a dQ workspace tile
 
 // Device workspace of a backward call (all fp32):
-//   dq   [B*Hq][ntq][d_qk][128]   dQ accumulator, each 128-row tile stored
-//                                 column by column (row fastest)
+//   dq   [B*Hq][ntq][d_qk/4][128][4]  dQ accumulator: in each 128-row tile,
+//                                 groups of four columns, row by row
 //   nl2  [B*Hq][ntq*128]          -LSE * log2(e) (-inf for a row with no key
 //                                 and for padding rows)
 //   D    [B*Hq][ntq*128]          rowsum(dO * O) (0 for padding rows)
@@ -148,10 +148,12 @@ struct QWalk {
   }
 };
 
-// Index of dQ element (row t, column c) of head bh in the workspace.
+// Index of dQ element (row t, column c) of head bh in the workspace.  A
+// 128-row tile is stored as [c / 4][row][c % 4]: four consecutive columns of
+// a row are one 16-byte vector and 32 consecutive rows 512 contiguous bytes.
 __device__ __forceinline__ long long bwd_dq_index(const BwdArgs& a, int bh, int t, int c, int dqk) {
-  return ((static_cast<long long>(bh) * a.ntq_ws + t / kBwdTile) * dqk + c) * kBwdTile +
-         (t % kBwdTile);
+  return (((static_cast<long long>(bh) * a.ntq_ws + t / kBwdTile) * (dqk / 4) + c / 4) *
+              kBwdTile + (t % kBwdTile)) * 4 + (c % 4);
 }
 
 }  // namespace ra

@@ -6,16 +6,18 @@
 // persistent; work item = one 128-key tile of one (batch, KV head)):
 //   warp 0      TMA producer: K, V of the item; then per visit Q, dO (TMA) and
 //               the visit's -LSE log2(e) and D vectors (bulk copies), two stages
-//   warp 1      tcgen05.mma issuer; owns the tensor-memory allocation
-//   warps 2-3   idle
-//   warps 4-7   "compute": thread r owns key r of the tile (TMEM lane r):
-//               P^T = 2^(scale log2(e) S^T - LSE log2(e)) into TMEM as bf16,
-//               then dS^T = P^T (dP^T - D) into shared memory as bf16
-//   warps 8-11  "reduce": reads each visit's dQ tile out of TMEM and adds it
-//               into the fp32 workspace (red.add, a warp covers 32 consecutive
-//               floats); at the end of the item writes dK, dV
-// Registers: launched at 168 per thread; setmaxnreg moves them to 224
-// (compute) + 160 (reduce) + 120 (producer / MMA warpgroup) = 504 = 3 x 168.
+//   warps 1-3   tcgen05.mma issuers (three, see below); warp 1 owns the
+//               tensor-memory allocation
+//   warps 4-11  "compute", two warpgroups, query columns 0-63 and 64-127:
+//               thread r owns key r of the tile (TMEM lane r) and forms
+//               P^T = 2^(scale log2(e) S^T - LSE log2(e)) (into TMEM as bf16)
+//               and dS^T = P^T (dP^T - D) (into shared memory as bf16) for
+//               its half; between the two it reads the previous visit's dQ
+//               (its half of the columns, lane r = query r) out of TMEM and
+//               adds it into the fp32 workspace with 16-byte vector
+//               reductions; at the end of the item it writes its half of dK, dV
+// Registers: launched at 168 per thread; setmaxnreg moves them to 2 x 184
+// (compute) + 136 (producer / MMA warpgroup) = 504 = 3 x 168.
 //
 // Per visit (query tile t of head h against the item's key tile):
 //   S^T  = K Q_t^T        M = 128 keys, N = 128 queries   (A, B K-major)
@@ -30,12 +32,11 @@
 // Tensor memory (512 columns): S^T [0,128) (P^T packed over its first 64
 // columns), dP^T [128,256) (dQ over it once the compute warps have loaded
 // dP^T), dV [256,256+DV), dK [256+DV,256+DV+DQK).
-// MMA issue order per visit v: dV(v), S^T(v+1), dK(v), dQ(v), dP^T(v+1).
-// MMAs of one thread execute in issue order, so S^T(v+1) overwrites P^T(v)
-// only after dV(v) has read it, and the compute warps form P^T(v+1) while the
-// tensor cores run dK(v) and dQ(v).  A commit fires when every MMA issued
-// before it has completed: dP^T(v+1)'s also tells the compute warps that
-// dK(v) and dQ(v) are done with the dS tile.
+// Products per visit v and their issuers: A issues dV(v) then S^T(v+1), B
+// issues dK(v), C issues dQ(v) then dP^T(v+1).  MMAs of one thread execute
+// in issue order, so S^T(v+1) overwrites P^T(v) only after dV(v) has read it
+// and dP^T(v+1) overwrites dQ(v) only after it was read out; the compute
+// warps form P^T(v+1) while the tensor cores run dK(v) and dQ(v).
 #include <cuda.h>
 
 #include "block_class.cuh"
@@ -53,15 +54,13 @@ constexpr int kT = 128;
 constexpr int kBox = 128 * 64 * 2;  // TMA box: 128 rows x 64 bf16
 constexpr int kThreads = 384;
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsCompute = 224;
-constexpr int kRegsReduce = 160;
-constexpr int kRegsOther = 120;
-static_assert(kRegsCompute + kRegsReduce + kRegsOther <= 3 * kRegsLaunch,
+constexpr int kRegsCompute = 184;
+constexpr int kRegsOther = 136;
+static_assert(2 * kRegsCompute + kRegsOther <= 3 * kRegsLaunch,
               "register split must fit the launch allocation");
 // setmaxnreg.inc may only raise a warpgroup's count and .dec only lower it.
-static_assert(kRegsCompute >= kRegsLaunch, "compute warpgroup grows (setmaxnreg.inc)");
-static_assert(kRegsReduce <= kRegsLaunch && kRegsOther <= kRegsLaunch,
-              "reduce and producer / MMA warpgroups shrink (setmaxnreg.dec)");
+static_assert(kRegsCompute >= kRegsLaunch, "compute warpgroups grow (setmaxnreg.inc)");
+static_assert(kRegsOther <= kRegsLaunch, "producer / MMA warpgroup shrinks (setmaxnreg.dec)");
 constexpr int kSmemLimit = 232448;
 
 template <int DQK, int DV>
@@ -154,13 +153,15 @@ __device__ __forceinline__ void mma_mm(uint32_t d, uint32_t a, uint32_t b, uint3
     umma_ss(d, da + mnmaj_step(ks), db + mnmaj_step(ks), idesc, ks > 0 ? 1u : 0u);
 }
 
-// dK or dV of the item's keys out of tensor memory: `mul` times the
-// accumulator, stored (ring: bf16) or added (block: fp32).  Warp-collective.
-template <int D>
+// W columns (from col0) of dK or dV of the item's keys out of tensor memory:
+// `mul` times the accumulator, stored (ring: bf16) or added (block: fp32) into
+// rows of width D.  Warp-collective.
+template <int D, int W>
 __device__ __forceinline__ void store_key_grad(uint32_t taddr, bool any, bool valid, float mul,
-                                               void* dst, long long krow, int block_mode) {
+                                               void* dst, long long krow, int col0,
+                                               int block_mode) {
 #pragma unroll
-  for (int c0 = 0; c0 < D; c0 += 32) {
+  for (int c0 = 0; c0 < W; c0 += 32) {
     float o[32];
     if (any) {
       tmem_ld32f(taddr + c0, o);
@@ -171,7 +172,7 @@ __device__ __forceinline__ void store_key_grad(uint32_t taddr, bool any, bool va
       for (int c = 0; c < 32; ++c) o[c] = 0.f;
     }
     if (valid && block_mode) {
-      float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + krow * D + c0);
+      float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + krow * D + col0 + c0);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         float4 x = d4[c];
@@ -182,7 +183,8 @@ __device__ __forceinline__ void store_key_grad(uint32_t taddr, bool any, bool va
         d4[c] = x;
       }
     } else if (valid) {
-      uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + krow * D + c0);
+      uint4* d4 =
+          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + krow * D + col0 + c0);
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         d4[c] = make_uint4(pack_bf16x2(o[8 * c] * mul, o[8 * c + 1] * mul),
@@ -226,7 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
   uint64_t* acc_full = bars + 12;
   uint64_t* acc_empty = bars + 13;
   uint64_t* drain = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* s_read = bars + 15;  // both compute halves hold their S^T
+  uint64_t* dk_done = bars + 16;  // dK(v) has read the dS tile
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* kv_issued = abort_flag + 1;
   volatile int* q_issued = abort_flag + 2;
@@ -236,20 +240,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 1);
+    mbar_init(kv_empty, 2);  // issuers A and C
     for (int s = 0; s < 2; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
+      mbar_init(&q_empty[s], 2);  // issuers A and B
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, kT);
-    mbar_init(ds_full, kT);
+    mbar_init(p_full, 2 * kT);
+    mbar_init(ds_full, 2 * kT);
     mbar_init(dq_full, 1);
-    mbar_init(dq_empty, kT);
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kT);
-    mbar_init(drain, 1);
+    mbar_init(dq_empty, 2 * kT);
+    mbar_init(acc_full, 2);  // issuers A (dV) and B (dK)
+    mbar_init(acc_empty, 2 * kT);
+    mbar_init(drain, 3);
+    mbar_init(s_read, 2 * kT);
+    mbar_init(dk_done, 1);
     *abort_flag = 0;
     *kv_issued = 0;
     *q_issued = 0;
@@ -304,12 +310,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
         } while (w.next(a, it, qt, h));
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer --
+  } else if (warp <= 3) {
+    // ------------------------------------------------------ MMA issuers --
+    // One thread issues tcgen05.mma at a limited rate, so three warps issue
+    // the visit's five products, each in an order that keeps its own
+    // overwrites safe (MMAs of one thread execute in issue order):
+    //   A (warp 1): dV(v), then S^T(v+1) over P^T(v), which dV(v) has read
+    //   B (warp 2): dK(v)
+    //   C (warp 3): dQ(v) over dP^T(v), then dP^T(v+1) once dQ(v) is read out
+    // A commit only covers its own thread's MMAs: barriers that speak for
+    // products of two issuers take one commit from each.
     if (lane == 0) {
-      uint32_t nkv = 0, nv = 0, nacc = 0;  // nv: visits so far = query-stage counter
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ);
       const uint32_t adO = smem_u32(sdO), adS = smem_u32(sdS);
+      uint32_t nkv = 0, nv = 0, nacc = 0;  // nv: visits so far = query-stage counter
       BItem it;
       bool ok = true;
       for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
@@ -317,107 +331,151 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
         w.start(a, it);
         int qt, h;
         if (!w.next(a, it, qt, h)) continue;
-        if (!(ok = mbar_wait(kv_full, nkv & 1, a.ctx, abort_flag))) break;
-        ++nkv;
-        tc_fence_after();
-        {  // S^T and dP^T of the item's first visit
+        if (warp != 2) {  // A and C read K, V
+          if (!(ok = mbar_wait(kv_full, nkv & 1, a.ctx, abort_flag))) break;
+          tc_fence_after();
+          ++nkv;
+        }
+        {
           const uint32_t st = nv & 1;
-          if (!(ok = mbar_wait(&q_full[st], (nv >> 1) & 1, a.ctx, abort_flag))) break;
-          tc_fence_after();
-          mma_kk<DQK>(tmem + C::S_COL, aK, aQ + st * C::QB * kBox, C::ID_S);
-          umma_commit(s_full);
-          // dP^T goes over the previous visit's dQ: wait until it is read out
-          if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
-          tc_fence_after();
-          mma_kk<DV>(tmem + C::DP_COL, aV, adO + st * C::VB * kBox, C::ID_S);
-          umma_commit(dp_full);
+          if (warp == 1) {  // S^T of the item's first visit
+            if (!(ok = mbar_wait(&q_full[st], (nv >> 1) & 1, a.ctx, abort_flag))) break;
+            tc_fence_after();
+            mma_kk<DQK>(tmem + C::S_COL, aK, aQ + st * C::QB * kBox, C::ID_S);
+            umma_commit(s_full);
+          } else if (warp == 3) {  // its dP^T, over the previous dQ once read out
+            if (!(ok = mbar_wait(&q_full[st], (nv >> 1) & 1, a.ctx, abort_flag))) break;
+            if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
+            tc_fence_after();
+            mma_kk<DV>(tmem + C::DP_COL, aV, adO + st * C::VB * kBox, C::ID_S);
+            umma_commit(dp_full);
+          }
         }
         bool first = true, has = true;
         while (has) {
           int nqt, nh;
           const bool has_next = w.next(a, it, nqt, nh);
           const uint32_t st = nv & 1, st1 = (nv + 1) & 1;
-          const uint32_t q_s = aQ + st * C::QB * kBox;
-          const uint32_t do_s = adO + st * C::VB * kBox;
-          if (!(ok = mbar_wait(p_full, nv & 1, a.ctx, abort_flag))) break;
-          tc_fence_after();
-          if (first) {  // the previous item's dK, dV have been read out
-            if (!(ok = mbar_wait(acc_empty, (nacc & 1) ^ 1, a.ctx, abort_flag))) break;
+          if (warp == 1) {
+            if (!(ok = mbar_wait(p_full, nv & 1, a.ctx, abort_flag))) break;
             tc_fence_after();
-          }
-          mma_tm(tmem + C::DV_COL, tmem + C::S_COL, do_s, C::ID_DV, !first);
-          if (has_next) {  // next S^T over P^T, which dV (issued before) has read
-            if (!(ok = mbar_wait(&q_full[st1], ((nv + 1) >> 1) & 1, a.ctx, abort_flag))) break;
+            if (first) {  // the previous item's dK, dV have been read out
+              if (!(ok = mbar_wait(acc_empty, (nacc & 1) ^ 1, a.ctx, abort_flag))) break;
+              tc_fence_after();
+            }
+            mma_tm(tmem + C::DV_COL, tmem + C::S_COL, adO + st * C::VB * kBox, C::ID_DV, !first);
+            umma_commit(&q_empty[st]);
+            if (has_next) {
+              if (!(ok = mbar_wait(&q_full[st1], ((nv + 1) >> 1) & 1, a.ctx, abort_flag))) break;
+              tc_fence_after();
+              mma_kk<DQK>(tmem + C::S_COL, aK, aQ + st1 * C::QB * kBox, C::ID_S);
+              umma_commit(s_full);
+            } else {
+              umma_commit(acc_full);
+              umma_commit(kv_empty);
+            }
+          } else if (warp == 2) {
+            if (!(ok = mbar_wait(ds_full, nv & 1, a.ctx, abort_flag))) break;
             tc_fence_after();
-            mma_kk<DQK>(tmem + C::S_COL, aK, aQ + st1 * C::QB * kBox, C::ID_S);
-            umma_commit(s_full);
-          }
-          if (!(ok = mbar_wait(ds_full, nv & 1, a.ctx, abort_flag))) break;
-          tc_fence_after();
-          mma_km(tmem + C::DK_COL, adS, q_s, C::ID_DK, !first);
-          mma_mm(tmem + C::DQ_COL, adS, aK, C::ID_DQ);  // dP^T was loaded before ds_full
-          umma_commit(dq_full);
-          umma_commit(&q_empty[st]);
-          if (!has_next) {
-            umma_commit(acc_full);
-            umma_commit(kv_empty);
-            ++nacc;
+            if (first) {
+              if (!(ok = mbar_wait(acc_empty, (nacc & 1) ^ 1, a.ctx, abort_flag))) break;
+              tc_fence_after();
+            }
+            mma_km(tmem + C::DK_COL, adS, aQ + st * C::QB * kBox, C::ID_DK, !first);
+            umma_commit(&q_empty[st]);
+            umma_commit(dk_done);
+            if (!has_next) umma_commit(acc_full);
+          } else {
+            if (!(ok = mbar_wait(ds_full, nv & 1, a.ctx, abort_flag))) break;
+            tc_fence_after();
+            mma_mm(tmem + C::DQ_COL, adS, aK, C::ID_DQ);  // dP^T(v) was loaded before ds_full
+            umma_commit(dq_full);
+            if (has_next) {
+              if (!(ok = mbar_wait(&q_full[st1], ((nv + 1) >> 1) & 1, a.ctx, abort_flag))) break;
+              if (!(ok = mbar_wait(dq_empty, nv & 1, a.ctx, abort_flag))) break;
+              tc_fence_after();
+              mma_kk<DV>(tmem + C::DP_COL, aV, adO + st1 * C::VB * kBox, C::ID_S);
+              umma_commit(dp_full);
+            } else {
+              umma_commit(kv_empty);
+            }
           }
           ++nv;
           first = false;
-          if (has_next) {  // next dP^T over this dQ, once it is read out
-            if (!(ok = mbar_wait(dq_empty, (nv & 1) ^ 1, a.ctx, abort_flag))) break;
-            tc_fence_after();
-            mma_kk<DV>(tmem + C::DP_COL, aV, adO + st1 * C::VB * kBox, C::ID_S);
-            umma_commit(dp_full);
-          }
           qt = nqt;
           h = nh;
           has = has_next;
         }
         if (!ok) break;
+        ++nacc;
       }
-      // every MMA issued so far has finished before the allocation goes away
+      // every MMA this thread issued has finished before the allocation goes away
       umma_commit(drain);
       const unsigned long long t0 = globaltimer_ns();
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < a.ctx.wait_ns) {
       }
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------------------------------------- compute: P^T and dS^T --
+  } else if (warp >= 4) {
+    // ------------------- compute: two warpgroups, 64 query columns each --
     regs_inc<kRegsCompute>();
-    const int row = threadIdx.x & 127;  // key of the tile = TMEM lane
+    const int half = (warp >> 2) - 1;  // 0: warps 4-7, 1: warps 8-11
+    const int row = threadIdx.x & 127;  // TMEM lane: key (S^T, dP^T, dK, dV), query (dQ)
     const uint32_t lb = tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
+    const int qc = half * 64;           // first query column of this warpgroup
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-    uint8_t* ds_row = sdS + row * 128;
+    uint8_t* ds_row = sdS + half * kBox + row * 128;  // atom `half`: queries qc .. qc+63
     const uint32_t sw = row & 7;
-    uint32_t nq = 0, nv = 0;
+    uint32_t nv = 0, nacc = 0;
     BItem it;
     bool ok = true;
+    // dQ of the latest visit, read out of tensor memory (over the dP^T
+    // columns) and added into the workspace: this half's DQK / 2 columns,
+    // 16-byte vector reductions, a warp covering 512 contiguous bytes
+    auto drain_dq = [&](int dq_bh, int dq_qt) -> bool {
+      if (!mbar_wait(dq_full, (nv - 1) & 1, a.ctx, abort_flag)) return false;
+      tc_fence_after();
+      float acc[DQK / 2];
+#pragma unroll
+      for (int c0 = 0; c0 < DQK / 2; c0 += 32)
+        tmem_ld32f(lb + C::DQ_COL + half * (DQK / 2) + c0, acc + c0);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c0 = 0; c0 < DQK / 2; c0 += 32) reg_fence32(acc + c0);
+      tc_fence_before();
+      mbar_arrive(dq_empty);
+      float* dst = a.ws_dq + bwd_dq_index(a, dq_bh, dq_qt * kT + row, half * (DQK / 2), DQK);
+#pragma unroll
+      for (int c = 0; c < DQK / 2; c += 4)
+        atomicAdd(reinterpret_cast<float4*>(dst + (c / 4) * (kT * 4)),
+                  make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+      return true;
+    };
     for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
       QWalk w;
       w.start(a, it);
       int qt, h;
+      int pend_bh = -1, pend_qt = 0;  // visit whose dQ is still in tensor memory
+      bool any = false;
       while (w.next(a, it, qt, h)) {
-        const int st = nq & 1;
-        if (!(ok = mbar_wait(&q_full[st], (nq >> 1) & 1, a.ctx, abort_flag))) break;
+        const int st = nv & 1;
+        if (!(ok = mbar_wait(&q_full[st], (nv >> 1) & 1, a.ctx, abort_flag))) break;
         if (!(ok = mbar_wait(s_full, nv & 1, a.ctx, abort_flag))) break;
         tc_fence_after();
-        const float* nl = vec + st * 2 * kT;
-        const float* dd = nl + kT;
-        float p[kT];
-        tmem_ld32f(lb + C::S_COL, p);
-        tmem_ld32f(lb + C::S_COL + 32, p + 32);
-        tmem_ld32f(lb + C::S_COL + 64, p + 64);
-        tmem_ld32f(lb + C::S_COL + 96, p + 96);
+        const float* nl = vec + st * 2 * kT + qc;
+        const float* dd = vec + st * 2 * kT + kT + qc;
+        float p[64];
+        tmem_ld32f(lb + C::S_COL + qc, p);
+        tmem_ld32f(lb + C::S_COL + qc + 32, p + 32);
         tmem_ld_wait();
         reg_fence32(p);
         reg_fence32(p + 32);
-        reg_fence32(p + 64);
-        reg_fence32(p + 96);
+        // P^T (packed, columns [0,64)) overwrites the S^T columns of queries
+        // 0-63: both halves must hold their S^T first (a bounded wait)
+        mbar_arrive(s_read);
+        if (!(ok = mbar_wait(s_read, nv & 1, a.ctx, abort_flag))) break;
         // p = 2^(s scale log2(e) - LSE log2(e)); padding rows carry -inf
 #pragma unroll
-        for (int c = 0; c < kT; c += 2) {
+        for (int c = 0; c < 64; c += 2) {
           const float2 n2 = *reinterpret_cast<const float2*>(nl + c);
           const float2 x = __ffma2_rn(make_float2(p[c], p[c + 1]), sc2, n2);
           p[c] = fast_exp2(x.x);
@@ -426,96 +484,72 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
         if (w.cls == kPartial || it.klen < kT) {
           // key `row` is visible to query column q iff q >= qmin
           long long qmin = 0;
-          if (a.causal)
-            qmin = row + it.k0 - w.q0 - floor_div(w.qoff - it.koff, a.stride);
+          if (a.causal) qmin = row + it.k0 - w.q0 - floor_div(w.qoff - it.koff, a.stride);
           if (row >= it.klen) qmin = kT;
-          const int qm = qmin < 0 ? 0 : (qmin > kT ? kT : static_cast<int>(qmin));
+          qmin -= qc;
+          const int qm = qmin < 0 ? 0 : (qmin > 64 ? 64 : static_cast<int>(qmin));
 #pragma unroll
-          for (int c = 0; c < kT; ++c)
+          for (int c = 0; c < 64; ++c)
             if (c < qm) p[c] = 0.f;
         }
 #pragma unroll
-        for (int c0 = 0; c0 < kT; c0 += 32) {
+        for (int c0 = 0; c0 < 64; c0 += 32) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) pk[c >> 1] = pack_bf16x2(p[c0 + c], p[c0 + c + 1]);
-          tmem_st16(lb + C::S_COL + (c0 >> 1), pk);
+          tmem_st16(lb + C::S_COL + ((qc + c0) >> 1), pk);
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
+        // the previous visit's dQ, while the tensor cores run dV and the next S^T
+        if (pend_bh >= 0 && !(ok = drain_dq(pend_bh, pend_qt))) break;
         if (!(ok = mbar_wait(dp_full, nv & 1, a.ctx, abort_flag))) break;
         tc_fence_after();
+        // the dS tile is free once dK(v-1) has read it (dQ(v-1) came before dP^T(v))
+        if (nv > 0 && !(ok = mbar_wait(dk_done, (nv - 1) & 1, a.ctx, abort_flag))) break;
         // dS^T = P^T (dP^T - D) -> bf16 rows of 64 queries, 128-byte swizzle
-#pragma unroll
-        for (int c0 = 0; c0 < kT; c0 += 64) {
+        {
           float dp[64];
-          tmem_ld32f(lb + C::DP_COL + c0, dp);
-          tmem_ld32f(lb + C::DP_COL + c0 + 32, dp + 32);
+          tmem_ld32f(lb + C::DP_COL + qc, dp);
+          tmem_ld32f(lb + C::DP_COL + qc + 32, dp + 32);
           tmem_ld_wait();
           reg_fence32(dp);
           reg_fence32(dp + 32);
-          uint8_t* atom = ds_row + (c0 / 64) * kBox;
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
             uint32_t w4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int c = g * 8 + e * 2;
-              const float2 d2 = *reinterpret_cast<const float2*>(dd + c0 + c);
-              w4[e] = pack_bf16x2(p[c0 + c] * (dp[c] - d2.x), p[c0 + c + 1] * (dp[c + 1] - d2.y));
+              const float2 d2 = *reinterpret_cast<const float2*>(dd + c);
+              w4[e] = pack_bf16x2(p[c] * (dp[c] - d2.x), p[c + 1] * (dp[c + 1] - d2.y));
             }
-            *reinterpret_cast<uint4*>(atom + ((g ^ sw) << 4)) =
+            *reinterpret_cast<uint4*>(ds_row + ((g ^ sw) << 4)) =
                 make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(ds_full);
-        ++nv;
-        ++nq;
-      }
-    }
-  } else if (warp >= 8) {
-    // ----------------------------------------- reduce: dQ out, dK / dV out --
-    regs_dec<kRegsReduce>();
-    const int row = threadIdx.x & 127;
-    const uint32_t lb = tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
-    uint32_t nv = 0, nacc = 0;
-    BItem it;
-    bool ok = true;
-    for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
-      QWalk w;
-      w.start(a, it);
-      int qt, h;
-      bool any = false;
-      while (w.next(a, it, qt, h)) {
-        if (!(ok = mbar_wait(dq_full, nv & 1, a.ctx, abort_flag))) break;
-        tc_fence_after();
-        float acc[DQK];
-#pragma unroll
-        for (int c0 = 0; c0 < DQK; c0 += 32) tmem_ld32f(lb + C::DQ_COL + c0, acc + c0);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c0 = 0; c0 < DQK; c0 += 32) reg_fence32(acc + c0);
-        tc_fence_before();
-        mbar_arrive(dq_empty);
-        const int bh = it.b * a.Hq + h;
-        float* dst = a.ws_dq + (static_cast<long long>(bh) * a.ntq_ws + qt) * DQK * kT + row;
-#pragma unroll
-        for (int c = 0; c < DQK; ++c) atomicAdd(dst + c * kT, acc[c]);
+        pend_bh = it.b * a.Hq + h;
+        pend_qt = qt;
         ++nv;
         any = true;
       }
       if (!ok) break;
+      if (pend_bh >= 0 && !(ok = drain_dq(pend_bh, pend_qt))) break;
+      // ---- dK, dV of the key tile: this half's columns ----
       if (any) {
         if (!(ok = mbar_wait(acc_full, nacc & 1, a.ctx, abort_flag))) break;
         tc_fence_after();
       }
       const bool valid = row < it.klen;
       const long long krow = static_cast<long long>(it.bkv) * a.n_k + it.k0 + row;
-      store_key_grad<DV>(lb + C::DV_COL, any, valid, 1.f, a.dv, krow, a.block_mode);
-      store_key_grad<DQK>(lb + C::DK_COL, any, valid, a.scale, a.dk, krow, a.block_mode);
+      store_key_grad<DV, DV / 2>(lb + C::DV_COL + half * (DV / 2), any, valid, 1.f, a.dv, krow,
+                                 half * (DV / 2), a.block_mode);
+      store_key_grad<DQK, DQK / 2>(lb + C::DK_COL + half * (DQK / 2), any, valid, a.scale, a.dk,
+                                   krow, half * (DQK / 2), a.block_mode);
       if (any) {
         tc_fence_before();
         mbar_arrive(acc_empty);
@@ -611,7 +645,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(PrepArgs p) {
 // dQ = scale * workspace (ring: stored in the output dtype) or dQ += scale *
 // workspace (block: fp32 accumulator).  One CTA per (head, 128-row tile); 32
 // columns at a time pass through shared memory to turn the workspace's
-// column-major tile into row-major rows.
+// [column / 4][row][column % 4] tile into row-major rows.
 template <typename T, bool ACCUM>
 __global__ void __launch_bounds__(256) bwd_dq_finalize_kernel(const float* ws, T* dq, float scale,
                                                               int n_q, int d_qk, int ntq) {
@@ -621,8 +655,9 @@ __global__ void __launch_bounds__(256) bwd_dq_finalize_kernel(const float* ws, T
   const float* src = ws + (bh * ntq + qt) * static_cast<long long>(d_qk) * kT;
   const int t0 = qt * kT;
   for (int c0 = 0; c0 < d_qk; c0 += 32) {
+    // columns c0 .. c0+31 are 8 groups of [128 rows][4], 4096 contiguous floats
     for (int i = threadIdx.x; i < 32 * kT; i += blockDim.x)
-      tile[i / kT][i % kT] = src[static_cast<long long>(c0) * kT + i];
+      tile[(i >> 9) * 4 + (i & 3)][(i >> 2) & (kT - 1)] = src[static_cast<long long>(c0) * kT + i];
     __syncthreads();
     for (int i = threadIdx.x; i < 32 * kT; i += blockDim.x) {
       const int r = i / 32, c = i % 32;
