@@ -105,9 +105,10 @@ def attention_backward_sampled(q, k, v, do, scale: float, causal: bool, rows, ke
     """The same gradients at a sample: dQ at query ``rows`` of query ``heads``,
     dK and dV at ``keys`` of ``kv_heads`` (positions 0..n-1, n_q == n_k).
 
-    dQ_t needs only row t; dK_u, dV_u need column u of every row, i.e. every
-    row's LSE and D, which come from ``oracle.attention.attention`` over all
-    rows.  Returns dq [B, len(heads), len(rows), dqk],
+    dQ_t needs only row t; dK_u, dV_u need column u of every row that sees
+    key u (every row, or with a causal mask the rows t >= u), i.e. those
+    rows' LSE and D, which come from ``oracle.attention.attention`` over just
+    those rows.  Returns dq [B, len(heads), len(rows), dqk],
     dk [B, len(kv_heads), len(keys), dqk], dv [B, len(kv_heads), len(keys), dv].
     """
     B, h_q, n, dqk = q.shape
@@ -122,13 +123,21 @@ def attention_backward_sampled(q, k, v, do, scale: float, causal: bool, rows, ke
     dq = np.zeros((B, len(heads), len(rows), dqk))
     dk = np.zeros((B, len(kv_heads), len(keys), dqk))
     dv = np.zeros((B, len(kv_heads), len(keys), dvd))
-    need_all = sorted(set(heads) | {g * grp + r for g in kv_heads for r in range(grp)})
+    need_heads = sorted(set(heads) | {g * grp + r for g in kv_heads for r in range(grp)})
+    # rows whose statistics are needed: the sampled rows, plus every row that
+    # can see a sampled key
+    tail = np.arange(int(keys.min()) if (causal and len(keys)) else 0, n, dtype=np.int64)
+    need_rows = np.union1d(rows, tail if len(keys) else np.zeros(0, np.int64))
     for b in range(B):
         stats = {}
-        for h in need_all:
-            o, lse = attention(q[b:b + 1], k[b:b + 1], v[b:b + 1], scale, causal,
-                               heads=[h], row_chunk=row_chunk)
-            stats[h] = (lse[0, 0], (o[0, 0] * _as_f64(do[b, h])).sum(axis=1))
+        for h in need_heads:
+            o, lse_r = attention(q[b:b + 1], k[b:b + 1], v[b:b + 1], scale, causal,
+                                 heads=[h], rows=need_rows, row_chunk=row_chunk)
+            lse = np.full(n, np.nan)
+            dlt = np.full(n, np.nan)
+            lse[need_rows] = lse_r[0, 0]
+            dlt[need_rows] = (o[0, 0] * _as_f64(do[b, h][need_rows])).sum(axis=1)
+            stats[h] = (lse, dlt)
         for hi, h in enumerate(heads):
             g = h // grp
             kk, vv = _as_f64(k[b, g]), _as_f64(v[b, g])
@@ -146,11 +155,11 @@ def attention_backward_sampled(q, k, v, do, scale: float, causal: bool, rows, ke
             kc, vc = _as_f64(k[b, g][keys]), _as_f64(v[b, g][keys])
             for r in range(grp):
                 h = g * grp + r
-                qa, doa = _as_f64(q[b, h]), _as_f64(do[b, h])
-                lse, dlt = stats[h]
-                st = (qa @ kc.T) * scale                      # [n, len(keys)]
+                qa, doa = _as_f64(q[b, h][tail]), _as_f64(do[b, h][tail])
+                lse, dlt = stats[h][0][tail], stats[h][1][tail]
+                st = (qa @ kc.T) * scale                      # [len(tail), len(keys)]
                 if causal:
-                    st = np.where(keys[None, :] <= pos[:, None], st, -np.inf)
+                    st = np.where(keys[None, :] <= tail[:, None], st, -np.inf)
                 live = np.isfinite(lse)
                 p = np.zeros_like(st)
                 p[live] = np.exp(st[live] - lse[live, None])

@@ -12,6 +12,9 @@ kernel at a shape the bench uses, holding at most a few GB on the device:
                  1M-token cache (B = 4, 64/8 heads): one chunk-kernel launch
                  and one merge launch, as one shard of the bench's decode step
   merge_p8       LSE merge of 8 fp32 partials of shape [1, 32, 16384, 128]
+  backward_cfg2  ring backward (prep, tensor-core kernel, dQ conversion) on the
+                 bench's default workload, from its own forward O and LSE
+  backward_gqa32k ring backward, causal GQA 32/8 heads, n = 32768, P = 8
 """
 from __future__ import annotations
 
@@ -20,7 +23,7 @@ import argparse
 import torch
 
 from . import ra
-from .workloads import make_qkv, make_workload_inputs, workload
+from .workloads import make_dout, make_qkv, make_workload_inputs, workload
 
 
 def _prefill(q, k, v, P, reps):
@@ -31,9 +34,20 @@ def _prefill(q, k, v, P, reps):
     torch.cuda.synchronize()
 
 
+def _backward(q, k, v, P, reps):
+    g = make_dout(q.shape[0], q.shape[1], q.shape[2], v.shape[-1], q.dtype, seed=9, device=q.device)
+    out, lse = ra.ring_forward(q, k, v, P, True)
+    ws = torch.empty(ra.backward_workspace_bytes(q, k, v), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for _ in range(2 + reps):
+        ra.ring_backward(q, k, v, out, lse, g, P, True, None, dq, dk, dv, ws)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["prefill_cfg2", "prefill_gqa32k", "decode_shard", "merge_p8"])
+    ap.add_argument("case", choices=["prefill_cfg2", "prefill_gqa32k", "decode_shard", "merge_p8",
+                                     "backward_cfg2", "backward_gqa32k"])
     ap.add_argument("--reps", type=int, default=1)
     args = ap.parse_args()
     dev = "cuda"
@@ -44,6 +58,13 @@ def main():
     elif args.case == "prefill_gqa32k":
         q, k, v = make_qkv(1, 32, 8, 32768, 32768, 128, 128, torch.bfloat16, seed=3, device=dev)
         _prefill(q, k, v, 8, args.reps)
+    elif args.case == "backward_cfg2":
+        wl = workload(2)
+        q, k, v = make_workload_inputs(wl, device=dev)
+        _backward(q, k, v, wl.P, args.reps)
+    elif args.case == "backward_gqa32k":
+        q, k, v = make_qkv(1, 32, 8, 32768, 32768, 128, 128, torch.bfloat16, seed=3, device=dev)
+        _backward(q, k, v, 8, args.reps)
     elif args.case == "decode_shard":
         q, k, v = make_qkv(4, 64, 8, 1, 131072, 128, 128, torch.bfloat16, seed=4, device=dev)
         ws = torch.empty(ra.decode_workspace_bytes(4, 64, 8, 131072), dtype=torch.uint8, device=dev)

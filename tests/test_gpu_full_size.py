@@ -83,3 +83,44 @@ def test_config4_decode_pass_q_1m():
         check_lse(lse[b:b + 1, heads], want_l[:, :, 0], f"LSE b={b} g={g}")
     del q, k, v
     torch.cuda.empty_cache()
+
+
+def test_config3_backward_gqa_128k():
+    # The ring backward on the causal GQA 128K workload in the bench's
+    # configuration: exact gradients on sampled query rows (dQ) and on the
+    # last 256 keys (dK, dV; a causal key u needs only rows t >= u), for the
+    # heads of two KV groups; identities over every key of every head:
+    # sum_u dK_u = 0 and sum_u dV_u = sum_t dO_t (per column).
+    from oracle.backward import attention_backward_sampled
+    from ring_context_parallelism_ra_b200.workloads import make_dout
+    from tests.parity_util import check_grad, to64
+    wl = workload(3)
+    torch.cuda.empty_cache()
+    q, k, v = make_workload_inputs(wl, device="cuda")
+    g = make_dout(wl.B, wl.Hq, wl.n, wl.d_v, wl.torch_dtype, seed=wl.seed, device="cuda")
+    out, lse = ra.ring_forward(q, k, v, wl.P, wl.causal, wl.scale)
+    dq, dk, dv = ra.ring_backward(q, k, v, out, lse, g, wl.P, wl.causal, wl.scale)
+    assert ra.get_status() == ra.RA_OK
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t).all().item()
+    G = wl.Hq // wl.Hkv
+    rows = sample_rows(wl.n, wl.P, n_uniform=24, seed=33)
+    keys = np.arange(wl.n - 256, wl.n)
+    for grp in (0, wl.Hkv - 1):
+        heads = list(range(grp * G, (grp + 1) * G))
+        q_s, g_s = q[:, heads].cpu(), g[:, heads].cpu()
+        k_s, v_s = k[:, grp:grp + 1].cpu(), v[:, grp:grp + 1].cpu()
+        wq, wk, wv = attention_backward_sampled(q_s, k_s, v_s, g_s, wl.scale, True, rows, keys)
+        ri = torch.as_tensor(rows, device="cuda")
+        ki = torch.as_tensor(keys, device="cuda")
+        check_grad(dq[:, heads][:, :, ri], wq, "bf16", "dQ sampled rows")
+        check_grad(dk[:, grp:grp + 1][:, :, ki], wk, "bf16", "dK last keys")
+        check_grad(dv[:, grp:grp + 1][:, :, ki], wv, "bf16", "dV last keys")
+    dk64 = dk.double()
+    dv64 = dv.double()
+    sk = dk64.sum(dim=2).abs()
+    assert (sk <= 2e-2 * (dk64 ** 2).sum(dim=2).sqrt()).all().item()
+    want_sv = g.double().reshape(wl.B, wl.Hkv, G, wl.n, wl.d_v).sum(dim=(2, 3))
+    assert ((dv64.sum(dim=2) - want_sv).abs() <= 2e-2 * (dv64 ** 2).sum(dim=2).sqrt()).all().item()
+    del q, k, v, g, out, lse, dq, dk, dv, dk64, dv64
+    torch.cuda.empty_cache()

@@ -206,3 +206,15 @@ def test_sampled_gradients_equal_whole_backward(causal):
     assert np.abs(sq - dq[:, [3, 0]][:, :, rows]).max() <= 1e-12
     assert np.abs(sk - dk[:, [1]][:, :, keys]).max() <= 1e-12
     assert np.abs(sv - dv[:, [1]][:, :, keys]).max() <= 1e-12
+
+
+def test_sampled_gradients_of_late_keys_use_only_later_rows():
+    # With a causal mask, dK_u and dV_u of late keys need only rows t >= u;
+    # the restricted computation must equal the whole backward.
+    q, k, v, g = _inputs(41, B=1, hq=4, hkv=2, nq=50, nk=50, d=6, dv=5)
+    dq, dk, dv = attention_backward(q, k, v, g, 0.4, True)
+    rows, keys = [3, 44], [49, 40, 45]
+    sq, sk, sv = attention_backward_sampled(q, k, v, g, 0.4, True, rows, keys)
+    assert np.abs(sq - dq[:, :, rows]).max() <= 1e-12
+    assert np.abs(sk - dk[:, :, keys]).max() <= 1e-12
+    assert np.abs(sv - dv[:, :, keys]).max() <= 1e-12
