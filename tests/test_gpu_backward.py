@@ -208,9 +208,14 @@ def test_backward_sampled_at_8k_mha_workload():
     check_grad(dk[:, :, sample], wk, "bf16", "dK sampled keys")
     check_grad(dv[:, :, sample], wv, "bf16", "dV sampled keys")
     # identities over every key (per column): sum_u dK_u = 0 and
-    # sum_u dV_u = sum_t dO_t; rounding errors of the n terms add up like a
-    # random walk, so the bar is relative to the terms' root sum of squares
+    # sum_u dV_u = sum_t dO_t.  Bar for a sum of n entries each within the
+    # element-wise bars: a systematic relative error (<= the bf16 mean bar,
+    # 2e-3) adds up to 2e-3 * sum |x|, random rounding to a root sum of squares
     dk64, dv64 = to64(dk), to64(dv)
-    assert (np.abs(dk64.sum(axis=2)) <= 2e-2 * np.sqrt((dk64 ** 2).sum(axis=2))).all()
+
+    def bar(x):
+        return 2e-3 * np.abs(x).sum(axis=2) + 2e-2 * np.sqrt((x ** 2).sum(axis=2))
+
+    assert (np.abs(dk64.sum(axis=2)) <= bar(dk64)).all()
     want_sv = to64(g).reshape(wl.B, wl.Hkv, -1, wl.n, wl.d_v).sum(axis=(2, 3))
-    assert (np.abs(dv64.sum(axis=2) - want_sv) <= 2e-2 * np.sqrt((dv64 ** 2).sum(axis=2))).all()
+    assert (np.abs(dv64.sum(axis=2) - want_sv) <= bar(dv64)).all()

@@ -116,11 +116,17 @@ def test_config3_backward_gqa_128k():
         check_grad(dq[:, heads][:, :, ri], wq, "bf16", "dQ sampled rows")
         check_grad(dk[:, grp:grp + 1][:, :, ki], wk, "bf16", "dK last keys")
         check_grad(dv[:, grp:grp + 1][:, :, ki], wv, "bf16", "dV last keys")
+    # bar for a sum of n entries each within the element-wise bars: a
+    # systematic relative error (<= the bf16 mean bar, 2e-3) adds up to
+    # 2e-3 * sum |x|, random rounding to a root sum of squares
     dk64 = dk.double()
     dv64 = dv.double()
-    sk = dk64.sum(dim=2).abs()
-    assert (sk <= 2e-2 * (dk64 ** 2).sum(dim=2).sqrt()).all().item()
+
+    def bar(x):
+        return 2e-3 * x.abs().sum(dim=2) + 2e-2 * (x ** 2).sum(dim=2).sqrt()
+
+    assert (dk64.sum(dim=2).abs() <= bar(dk64)).all().item()
     want_sv = g.double().reshape(wl.B, wl.Hkv, G, wl.n, wl.d_v).sum(dim=(2, 3))
-    assert ((dv64.sum(dim=2) - want_sv).abs() <= 2e-2 * (dv64 ** 2).sum(dim=2).sqrt()).all().item()
+    assert ((dv64.sum(dim=2) - want_sv).abs() <= bar(dv64)).all().item()
     del q, k, v, g, out, lse, dq, dk, dv, dk64, dv64
     torch.cuda.empty_cache()
