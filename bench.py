@@ -347,6 +347,7 @@ def run_backward_leg(args, world, rank, wl, peaks, peaks_kind):
     flops = backward_flops(wl)
     achieved = flops / (ms_local * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tr = load_traffic(f"ring_backward:{wl.name}", BWD_FILES)
     del q, k, v, g, out, lse, ws, dq, dk, dv, flush
     torch.cuda.empty_cache()
     return {"workload": wl.name, "value": round(world * flops / (ms * 1e-3) / 1e12, 3),
@@ -356,11 +357,16 @@ def run_backward_leg(args, world, rank, wl, peaks, peaks_kind):
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peaks_kind} bf16 burst",
+                         "frac_of_sustained": round(
+                             achieved / peaks.get("bf16_tflops_sustained", 1400.0), 4),
+                         "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                         "traffic_kernel": "bwd_tc_kernel (ncu capture of the same shape)",
                          "kernel": "ring_backward (prep + tcgen05 kernel + dQ conversion)"},
             "clocks": clk.summary()}
 
 
 TC_FILES = ["tc_attention.cu", "ptx.cuh", "block_class.cuh"]
+BWD_FILES = ["bwd_attention.cu", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
 
 
 def run_striped_leg(args, world, rank, wl, peaks):
