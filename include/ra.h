@@ -243,7 +243,7 @@ size_t ra_backward_workspace_bytes(const ra_shape* shape);
  *   out, dout   : device [B, Hq, n_q, d_v] of shape->dtype (O of the forward
  *                 and the gradient arriving at it).
  *   delta       : device fp32 [B, Hq, n_q].
- * Errors: RA_ERR_INVALID, RA_ERR_CUDA.
+ * Errors: RA_ERR_INVALID, RA_ERR_UNSUPPORTED (d_v other than 64, 128), RA_ERR_CUDA.
  */
 int ra_backward_delta(const void* out, const void* dout, const ra_shape* shape, float* delta,
                       void* stream);

@@ -1,6 +1,7 @@
-// Backward pass of exact attention on the tensor cores (bf16 inputs), plus the
-// small kernels around it (row statistics in, dQ out) shared with the fp32
-// path.  What is computed is stated in bwd.cuh.
+// Backward pass of exact attention on the tensor cores (bf16 inputs) and the
+// launcher of the whole backward call (row statistics, the gradient kernel of
+// the input dtype, the dQ conversion).  What is computed is stated in bwd.cuh;
+// the row kernels are in bwd_rows.cu.
 //
 // CTA layout of the tensor-core kernel (384 threads, one CTA per SM,
 // persistent; work item = one 128-key tile of one (batch, KV head)):
@@ -583,98 +584,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// ------------------------------------------------------------- prep / out --
-
-struct PrepArgs {
-  const void* out;     // forward output (D = rowsum(dO * O)), or null
-  const void* dout;
-  const float* delta;  // caller's D, used when out is null
-  const float* lse;    // forward LSE, or null (delta-only mode)
-  int n_q, d_v;
-  int row_pitch;       // rows per head in the destination arrays
-  long long rows;      // B * Hq * row_pitch
-  float* nl2;          // [rows] or null
-  float* d_ws;         // [rows] or null
-  float* dq_ws;        // zeroed when non-null
-  long long dq_floats;
-  float* delta_out;    // [B * Hq * n_q] or null
-};
-
-// One warp per destination row.
-template <typename T>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(PrepArgs p) {
-  const int wpb = blockDim.x >> 5;
-  const long long nw = static_cast<long long>(gridDim.x) * wpb;
-  const long long gw = static_cast<long long>(blockIdx.x) * wpb + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  for (long long r = gw; r < p.rows; r += nw) {
-    const long long bh = r / p.row_pitch;
-    const int t = static_cast<int>(r % p.row_pitch);
-    float dsum = 0.f, nl = -INFINITY;
-    if (t < p.n_q) {
-      const long long src = bh * p.n_q + t;
-      if (p.out != nullptr) {
-        const T* o = static_cast<const T*>(p.out) + src * p.d_v;
-        const T* g = static_cast<const T*>(p.dout) + src * p.d_v;
-        for (int c = lane; c < p.d_v; c += 32) dsum += to_f32(o[c]) * to_f32(g[c]);
-#pragma unroll
-        for (int s = 16; s > 0; s >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, s);
-      } else {
-        dsum = p.delta[src];
-      }
-      if (p.lse != nullptr) {
-        const float l = p.lse[src];
-        nl = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
-      }
-    }
-    if (lane == 0) {
-      if (p.d_ws) p.d_ws[r] = dsum;
-      if (p.nl2) p.nl2[r] = nl;
-      if (p.delta_out && t < p.n_q) p.delta_out[bh * p.n_q + t] = dsum;
-    }
-  }
-  if (p.dq_ws != nullptr) {
-    float4* z = reinterpret_cast<float4*>(p.dq_ws);
-    const long long n4 = p.dq_floats / 4;
-    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
-         i += static_cast<long long>(gridDim.x) * blockDim.x)
-      z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-
-// dQ = scale * workspace (ring: stored in the output dtype) or dQ += scale *
-// workspace (block: fp32 accumulator).  One CTA per (head, 128-row tile); 32
-// columns at a time pass through shared memory to turn the workspace's
-// [column / 4][row][column % 4] tile into row-major rows.
-template <typename T, bool ACCUM>
-__global__ void __launch_bounds__(256) bwd_dq_finalize_kernel(const float* ws, T* dq, float scale,
-                                                              int n_q, int d_qk, int ntq) {
-  __shared__ float tile[32][kT + 1];
-  const long long bh = blockIdx.x / ntq;
-  const int qt = blockIdx.x % ntq;
-  const float* src = ws + (bh * ntq + qt) * static_cast<long long>(d_qk) * kT;
-  const int t0 = qt * kT;
-  for (int c0 = 0; c0 < d_qk; c0 += 32) {
-    // columns c0 .. c0+31 are 8 groups of [128 rows][4], 4096 contiguous floats
-    for (int i = threadIdx.x; i < 32 * kT; i += blockDim.x)
-      tile[(i >> 9) * 4 + (i & 3)][(i >> 2) & (kT - 1)] = src[static_cast<long long>(c0) * kT + i];
-    __syncthreads();
-    for (int i = threadIdx.x; i < 32 * kT; i += blockDim.x) {
-      const int r = i / 32, c = i % 32;
-      if (t0 + r < n_q) {
-        T* d = dq + (bh * n_q + t0 + r) * d_qk + c0 + c;
-        const float x = tile[c][r] * scale;
-        if constexpr (ACCUM) {
-          *d = *d + x;
-        } else {
-          *d = from_f32<T>(x);
-        }
-      }
-    }
-    __syncthreads();
-  }
-}
-
 template <int DQK, int DV>
 int launch_bwd_typed(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& tdo, const BwdArgs& args, int grid, cudaStream_t stream) {
@@ -690,35 +599,10 @@ int launch_bwd_typed(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
-int launch_prep(const PrepArgs& p, ra_dtype dt, const DeviceInfo& dev, cudaStream_t st) {
-  const long long blocks_rows = (p.rows + 7) / 8;
-  long long blocks = blocks_rows < 4LL * dev.num_sms ? blocks_rows : 4LL * dev.num_sms;
-  if (blocks < 1) blocks = 1;
-  if (dt == RA_BF16)
-    bwd_prep_kernel<__nv_bfloat16><<<static_cast<int>(blocks), 256, 0, st>>>(p);
-  else
-    bwd_prep_kernel<float><<<static_cast<int>(blocks), 256, 0, st>>>(p);
-  note_launch();
-  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
-}
-
 }  // namespace
 
 size_t backward_workspace_bytes(const ra_shape& s) {
   return bwd_layout(s.B, s.Hq, s.n_q, s.d_qk).total;
-}
-
-int launch_backward_delta(const void* out, const void* dout, const ra_shape& s, float* delta,
-                          const DeviceInfo& dev, cudaStream_t stream) {
-  PrepArgs p{};
-  p.out = out;
-  p.dout = dout;
-  p.n_q = s.n_q;
-  p.d_v = s.d_v;
-  p.row_pitch = s.n_q;
-  p.rows = static_cast<long long>(s.B) * s.Hq * s.n_q;
-  p.delta_out = delta;
-  return launch_prep(p, s.dtype, dev, stream);
 }
 
 int launch_backward(const void* q, const void* k, const void* v, const void* out,
@@ -732,20 +616,8 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
   float* ws_nl2 = reinterpret_cast<float*>(ws + L.nl2_off);
   float* ws_d = reinterpret_cast<float*>(ws + L.d_off);
 
-  PrepArgs p{};
-  p.out = block_mode ? nullptr : out;
-  p.dout = dout;
-  p.delta = delta;
-  p.lse = lse;
-  p.n_q = s.n_q;
-  p.d_v = s.d_v;
-  p.row_pitch = L.ntq * kBwdTile;
-  p.rows = L.rows_pad;
-  p.nl2 = ws_nl2;
-  p.d_ws = ws_d;
-  p.dq_ws = ws_dq;
-  p.dq_floats = L.rows_pad * s.d_qk;
-  int rc = launch_prep(p, s.dtype, dev, stream);
+  int rc = launch_backward_rows(block_mode ? nullptr : out, dout, delta, lse, s, L, ws_nl2, ws_d,
+                                ws_dq, dev, stream);
   if (rc != RA_OK) return rc;
 
   BwdArgs a{};
@@ -802,20 +674,7 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
   }
   if (rc != RA_OK) return rc;
 
-  const long long blocks = static_cast<long long>(s.B) * s.Hq * L.ntq;
-  if (blocks > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
-  if (block_mode) {
-    bwd_dq_finalize_kernel<float, true><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        ws_dq, static_cast<float*>(dq), scale, s.n_q, s.d_qk, L.ntq);
-  } else if (s.dtype == RA_BF16) {
-    bwd_dq_finalize_kernel<__nv_bfloat16, false><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        ws_dq, static_cast<__nv_bfloat16*>(dq), scale, s.n_q, s.d_qk, L.ntq);
-  } else {
-    bwd_dq_finalize_kernel<float, false><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        ws_dq, static_cast<float*>(dq), scale, s.n_q, s.d_qk, L.ntq);
-  }
-  note_launch();
-  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+  return launch_dq_finalize(ws_dq, dq, s, L, scale, block_mode, stream);
 }
 
 }  // namespace ra

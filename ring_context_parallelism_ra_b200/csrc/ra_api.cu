@@ -338,6 +338,7 @@ int ra_backward_delta(const void* out, const void* dout, const ra_shape* shape, 
   if (rc != RA_OK) return rc;
   if (!out || !dout || !delta) return RA_ERR_INVALID;
   if (!aligned16(out) || !aligned16(dout) || !aligned16(delta)) return RA_ERR_INVALID;
+  if (shape->d_v != 64 && shape->d_v != 128) return RA_ERR_UNSUPPORTED;
   DeviceInfo dev;
   rc = device_info(&dev);
   if (rc != RA_OK) return rc;

@@ -145,6 +145,7 @@ def test_backward_validation_rejects_bad_arguments_before_launch():
     assert blk(s, wsb=ctypes.c_size_t(0)) == INV
     assert L.ra_backward_delta(nul, p, ctypes.byref(s), p, nul) == INV
     assert L.ra_backward_delta(p, p, None, p, nul) == INV
+    assert L.ra_backward_delta(p, p, ctypes.byref(_shape(d_v=32)), p, nul) == UNS
 
 
 def test_backward_workspace_size():
