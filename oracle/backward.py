@@ -41,7 +41,7 @@ from .attention import _as_f64, attention, gqa_group
 from .blockwise import partition_bounds, ring_order
 
 __all__ = ["attention_backward", "attention_backward_sampled", "ring_attention_backward",
-           "row_delta"]
+           "block_backward_share", "row_delta"]
 
 
 def _positions(n, offset, positions):
@@ -166,6 +166,40 @@ def attention_backward_sampled(q, k, v, do, scale: float, causal: bool, rows, ke
                 ds = p * (doa @ vc.T - dlt[:, None])
                 dk[b, gi] += scale * (ds.T @ qa)
                 dv[b, gi] += p.T @ doa
+    return dq, dk, dv
+
+
+def block_backward_share(q, k, v, do, lse, delta, scale: float, causal: bool, q_positions,
+                         k_positions):
+    """One block's share of the gradients (dQ, dK, dV) in fp64, formed against
+    the query rows' final LSE and D = rowsum(dO * O) (passed in), for query
+    rows at ``q_positions`` and keys at ``k_positions``: what a device of the
+    ring adds when KV_j reaches Q_i.  Shapes as ``attention_backward``; lse,
+    delta [B, H_q, n_q]."""
+    B, h_q, n_q, dqk = q.shape
+    h_kv = k.shape[1]
+    grp = gqa_group(h_q, h_kv)
+    qp = np.asarray(q_positions, dtype=np.int64)
+    kp = np.asarray(k_positions, dtype=np.int64)
+    lse, delta = _as_f64(lse), _as_f64(delta)
+    dq = np.zeros((B, h_q, n_q, dqk))
+    dk = np.zeros(k.shape[:3] + (dqk,))
+    dv = np.zeros(v.shape)
+    for b in range(B):
+        for h in range(h_q):
+            g = h // grp
+            qh, doh = _as_f64(q[b, h]), _as_f64(do[b, h])
+            kk, vv = _as_f64(k[b, g]), _as_f64(v[b, g])
+            s = (qh @ kk.T) * scale
+            if causal:
+                s = np.where(kp[None, :] <= qp[:, None], s, -np.inf)
+            live = np.isfinite(lse[b, h])
+            p = np.zeros_like(s)
+            p[live] = np.exp(s[live] - lse[b, h][live, None])
+            ds = p * (doh @ vv.T - delta[b, h][:, None])
+            dq[b, h] += scale * (ds @ kk)
+            dk[b, g] += scale * (ds.T @ qh)
+            dv[b, g] += p.T @ doh
     return dq, dk, dv
 
 

@@ -1,0 +1,196 @@
+"""Ring Attention across devices: one sequence partition per rank, the KV
+partitions passed around the ring.
+
+Method (pages cited by title and section): each device keeps its query
+partition Q_i and sends its KV partition to the next device while receiving
+the previous device's, so that after P - 1 exchanges every query partition
+has met every KV partition (page "AI 推理系列（十一）：Ring Attention 如何让
+多张 GPU 共同计算一条超长序列", section "KV 在 Ring 中如何流动"); the exchange of
+step s + 1 overlaps the block computation of step s (same page, section "通信
+很多，为什么仍然可能划算"; page "LLM长文本推理Ring Attention环形注意力机制实现与
+优化", section "Ring Attention实现代码与通信重叠").  The block partials are
+merged with the log-sum-exp rule at the end.  With a causal mask a contiguous
+split skips the blocks wholly in the future (and leaves the devices unevenly
+loaded); the striped split of the latter page's tuning section gives rank r
+the tokens r, r + P, r + 2P, ... so that every block is about half visible.
+
+Backward: KV_j travels together with its gradient accumulators dK_j, dV_j,
+which collect one share per query partition; dQ_i collects at its rank; a
+last hop returns every accumulator to its owner.
+
+Layout on every rank: q [B, Hq, L, d_qk], k [B, Hkv, L, d_qk], v [B, Hkv, L,
+d_v] with L = n / P tokens of its partition, in position order.  Rank r is
+partition r of the ring (ring order = rank order of the process group).
+
+Transports:
+  * ``NcclTransport`` -- device tensors exchanged with batched NCCL
+    send / recv; the process group's side stream runs the exchange while the
+    current stream runs the block kernel.
+  * ``HostTransport`` -- send / recv through host memory (a gloo process
+    group, or CPU tensors); the exchange is synchronous.
+
+The block arithmetic is a pluggable ``blocks`` object; ``KernelBlocks`` (the
+default) runs the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import ra
+
+__all__ = ["KernelBlocks", "NcclTransport", "HostTransport", "default_transport",
+           "ring_attention_forward", "ring_attention_backward", "partition_positions"]
+
+
+class KernelBlocks:
+    """Block arithmetic on the library's kernels (bf16 on tensor cores, fp32
+    exact)."""
+
+    def partial(self, q, k, v, q_offset, k_offset, stride, causal, scale, o, lse):
+        return ra.block_partial_strided(q, k, v, q_offset, k_offset, stride, causal, scale, o, lse)
+
+    def merge(self, o_parts, lse_parts, out_dtype):
+        return ra.lse_merge(o_parts, lse_parts, out_dtype)
+
+    def delta(self, out, dout):
+        return ra.backward_delta(out, dout)
+
+    def backward(self, q, k, v, dout, lse, delta, q_offset, k_offset, stride, causal, scale,
+                 dq_acc, dk_acc, dv_acc):
+        ra.block_backward(q, k, v, dout, lse, delta, q_offset, k_offset, stride, causal, scale,
+                          dq_acc, dk_acc, dv_acc)
+
+
+class _Done:
+    def wait(self):
+        return None
+
+
+class NcclTransport:
+    """Send to the next rank and receive from the previous one with batched
+    NCCL point-to-point operations (asynchronous)."""
+
+    def __init__(self, group=None):
+        self.group = group
+
+    def exchange(self, send, recv, nxt, prv):
+        ops = [dist.P2POp(dist.isend, t, nxt, self.group) for t in send]
+        ops += [dist.P2POp(dist.irecv, t, prv, self.group) for t in recv]
+        reqs = dist.batch_isend_irecv(ops)
+
+        class _Handle:
+            def wait(self_inner):
+                for r in reqs:
+                    r.wait()
+        return _Handle()
+
+
+class HostTransport:
+    """Send / recv through host memory (for a gloo process group).  Device
+    tensors are staged through CPU copies; the exchange completes before
+    ``exchange`` returns."""
+
+    def __init__(self, group=None):
+        self.group = group
+
+    def exchange(self, send, recv, nxt, prv):
+        me = dist.get_rank(self.group)
+        staged = [t.detach().to("cpu") for t in send]
+        bufs = [torch.empty(t.shape, dtype=t.dtype) for t in recv]
+        # even ranks send first, odd ranks receive first: no cycle of blocking sends
+        for t, b in zip(staged, bufs):
+            if me % 2 == 0:
+                dist.send(t, nxt, self.group)
+                dist.recv(b, prv, self.group)
+            else:
+                dist.recv(b, prv, self.group)
+                dist.send(t, nxt, self.group)
+        for b, t in zip(bufs, recv):
+            t.copy_(b)
+        return _Done()
+
+
+def default_transport(group=None):
+    """NCCL for an NCCL process group, host staging otherwise."""
+    backend = dist.get_backend(group)
+    return NcclTransport(group) if backend == "nccl" else HostTransport(group)
+
+
+def partition_positions(rank: int, P: int, L: int, striped: bool):
+    """(offset, stride) of partition `rank`: token of local row t is
+    offset + t * stride."""
+    return (rank, P) if striped else (rank * L, 1)
+
+
+def _ring(group):
+    P = dist.get_world_size(group)
+    i = dist.get_rank(group)
+    return P, i, (i + 1) % P, (i - 1) % P
+
+
+def ring_attention_forward(q, k, v, causal=True, scale=None, striped=False, group=None,
+                           transport=None, blocks=None):
+    """This rank's output (O_i [B, Hq, L, d_v] in q's dtype, LSE_i fp32
+    [B, Hq, L]) of exact attention over the whole sequence, its query
+    partition meeting every KV partition as they pass around the ring."""
+    P, i, nxt, prv = _ring(group)
+    transport = transport or default_transport(group)
+    blocks = blocks or KernelBlocks()
+    B, Hq, L, _ = q.shape
+    dv = v.shape[-1]
+    scale = q.shape[-1] ** -0.5 if scale is None else scale
+    o_parts = torch.empty((P, B, Hq, L, dv), device=q.device, dtype=torch.float32)
+    l_parts = torch.empty((P, B, Hq, L), device=q.device, dtype=torch.float32)
+    cur = [k.contiguous(), v.contiguous()]
+    nbuf = [torch.empty_like(cur[0]), torch.empty_like(cur[1])]
+    q_off, stride = partition_positions(i, P, L, striped)
+    used = 0
+    for s in range(P):
+        j = (i - s) % P
+        handle = transport.exchange(cur, nbuf, nxt, prv) if s < P - 1 else _Done()
+        k_off, _ = partition_positions(j, P, L, striped)
+        if not (causal and not striped and j > i):  # wholly in the future: skipped
+            blocks.partial(q, cur[0], cur[1], q_off, k_off, stride, causal, scale,
+                           o_parts[used], l_parts[used])
+            used += 1
+        handle.wait()
+        if s < P - 1:
+            cur, nbuf = nbuf, cur
+    return blocks.merge(o_parts[:used], l_parts[:used], q.dtype)
+
+
+def ring_attention_backward(q, k, v, out, lse, dout, causal=True, scale=None, striped=False,
+                            group=None, transport=None, blocks=None):
+    """This rank's gradients (dQ_i, dK_i, dV_i, in q's dtype) of
+    ``ring_attention_forward``; ``out`` and ``lse`` are its outputs here."""
+    P, i, nxt, prv = _ring(group)
+    transport = transport or default_transport(group)
+    blocks = blocks or KernelBlocks()
+    B, Hq, L, _ = q.shape
+    scale = q.shape[-1] ** -0.5 if scale is None else scale
+    delta = blocks.delta(out, dout)
+    dq = torch.zeros(q.shape, device=q.device, dtype=torch.float32)
+    kv = [k.contiguous(), v.contiguous()]
+    kv_buf = [torch.empty_like(kv[0]), torch.empty_like(kv[1])]
+    acc = [torch.zeros(k.shape, device=q.device, dtype=torch.float32),
+           torch.zeros(v.shape, device=q.device, dtype=torch.float32)]
+    acc_buf = [torch.empty_like(acc[0]), torch.empty_like(acc[1])]
+    q_off, stride = partition_positions(i, P, L, striped)
+    for s in range(P):
+        j = (i - s) % P
+        # K, V of the next step travel while this step computes; the
+        # accumulators can only leave once this step has added its share
+        handle = transport.exchange(kv, kv_buf, nxt, prv) if s < P - 1 else _Done()
+        k_off, _ = partition_positions(j, P, L, striped)
+        if not (causal and not striped and j > i):
+            blocks.backward(q, kv[0], kv[1], dout, lse, delta, q_off, k_off, stride, causal,
+                            scale, dq, acc[0], acc[1])
+        if P > 1:
+            transport.exchange(acc, acc_buf, nxt, prv).wait()
+            acc, acc_buf = acc_buf, acc
+        handle.wait()
+        if s < P - 1:
+            kv, kv_buf = kv_buf, kv
+    # after P accumulator hops every rank holds its own dK, dV
+    return dq.to(q.dtype), acc[0].to(k.dtype), acc[1].to(v.dtype)

@@ -1,0 +1,122 @@
+"""CPU tests of the multi-device ring (ring_context_parallelism_ra_b200/
+distributed.py) over gloo with world sizes 2 and 3.  The block arithmetic is
+supplied by the fp64 oracle (a test-only ``blocks`` object), so these tests
+check the ring's own logic: the exchange schedule, the causal skip of a
+contiguous split, the striped positions, the final merge, and the routing of
+the travelling gradient accumulators back to their owners.  Each rank's
+result is compared with the oracle's whole-sequence attention and gradients."""
+import datetime
+import os
+import socket
+import sys
+import traceback
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class OracleBlocks:
+    """Block arithmetic from the oracle, for CPU tensors."""
+
+    @staticmethod
+    def _pos(off, stride, n):
+        return off + stride * np.arange(n, dtype=np.int64)
+
+    def partial(self, q, k, v, q_offset, k_offset, stride, causal, scale, o, lse):
+        from oracle.attention import attention
+        oo, ll = attention(q, k, v, scale, causal,
+                           q_positions=self._pos(q_offset, stride, q.shape[2]),
+                           k_positions=self._pos(k_offset, stride, k.shape[2]))
+        o.copy_(torch.from_numpy(oo))
+        lse.copy_(torch.from_numpy(ll))
+
+    def merge(self, o_parts, lse_parts, out_dtype):
+        from oracle.merge import lse_merge
+        oo, ll = lse_merge(o_parts.double().numpy(), lse_parts.double().numpy())
+        return torch.from_numpy(oo).to(out_dtype), torch.from_numpy(ll).float()
+
+    def delta(self, out, dout):
+        from oracle.backward import row_delta
+        return torch.from_numpy(row_delta(out, dout))
+
+    def backward(self, q, k, v, dout, lse, delta, q_offset, k_offset, stride, causal, scale,
+                 dq_acc, dk_acc, dv_acc):
+        from oracle.backward import block_backward_share
+        a, b, c = block_backward_share(q, k, v, dout, lse, delta, scale, causal,
+                                       self._pos(q_offset, stride, q.shape[2]),
+                                       self._pos(k_offset, stride, k.shape[2]))
+        dq_acc += torch.from_numpy(a).to(dq_acc.dtype)
+        dk_acc += torch.from_numpy(b).to(dk_acc.dtype)
+        dv_acc += torch.from_numpy(c).to(dv_acc.dtype)
+
+
+def _rank_main(rank, world, port, striped, causal, errq):
+    import torch.distributed as dist
+
+    from oracle.attention import attention
+    from oracle.backward import attention_backward
+    from ring_context_parallelism_ra_b200.distributed import (HostTransport,
+                                                              ring_attention_backward,
+                                                              ring_attention_forward)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, Hq, Hkv, L, d, dv = 1, 4, 2, 8, 6, 5
+        n = L * world
+        rng = np.random.default_rng(1000 + world)
+        q = torch.from_numpy(rng.standard_normal((B, Hq, n, d)))
+        k = torch.from_numpy(rng.standard_normal((B, Hkv, n, d)))
+        v = torch.from_numpy(rng.standard_normal((B, Hkv, n, dv)))
+        g = torch.from_numpy(rng.standard_normal((B, Hq, n, dv)))
+        rows = (np.arange(rank, n, world) if striped
+                else np.arange(rank * L, (rank + 1) * L))
+        part = lambda x: x[:, :, rows].contiguous()  # noqa: E731
+        scale = 0.4
+        tr, blocks = HostTransport(), OracleBlocks()
+        out, lse = ring_attention_forward(part(q), part(k), part(v), causal, scale, striped,
+                                          transport=tr, blocks=blocks)
+        want_o, want_l = attention(q, k, v, scale, causal)
+        assert np.abs(out.numpy() - want_o[:, :, rows]).max() <= 1e-6
+        assert np.abs(lse.numpy() - want_l[:, :, rows]).max() <= 1e-5
+        dq, dk, dvv = ring_attention_backward(part(q), part(k), part(v), out, lse, part(g), causal,
+                                              scale, striped, transport=tr, blocks=blocks)
+        wq, wk, wv = attention_backward(q, k, v, g, scale, causal)
+        for got, w in ((dq, wq), (dk, wk), (dvv, wv)):
+            assert np.abs(got.numpy() - w[:, :, rows]).max() <= 1e-5 * max(1.0, np.abs(w).max())
+    except Exception:
+        errq.put((rank, traceback.format_exc()))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("striped,causal", [(False, True), (True, True), (False, False)])
+def test_ring_over_gloo_matches_whole_sequence(world, striped, causal):
+    ctx = mp.get_context("spawn")
+    errq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, striped, causal, errq))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    errs = []
+    while not errq.empty():
+        errs.append(errq.get())
+    assert not errs, errs
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]

@@ -218,3 +218,30 @@ def test_sampled_gradients_of_late_keys_use_only_later_rows():
     assert np.abs(sq - dq[:, :, rows]).max() <= 1e-12
     assert np.abs(sk - dk[:, :, keys]).max() <= 1e-12
     assert np.abs(sv - dv[:, :, keys]).max() <= 1e-12
+
+
+@pytest.mark.parametrize("striped", [False, True])
+def test_block_shares_sum_to_the_whole_gradient(striped):
+    # Shares of every (Q_i, KV_j) block against the final LSE and D add up to
+    # the whole-row gradients (contiguous and striped positions).
+    from oracle.backward import block_backward_share
+    n, P = 24, 3
+    L = n // P
+    q, k, v, g = _inputs(51, B=1, hq=4, hkv=2, nq=n, nk=n, d=5, dv=4)
+    o, lse = attention(q, k, v, 0.5, True)
+    dlt = row_delta(o, g)
+    want = attention_backward(q, k, v, g, 0.5, True)
+    pos = lambda r: (np.arange(r, n, P) if striped else np.arange(r * L, (r + 1) * L))  # noqa: E731
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    for i in range(P):
+        for j in range(P):
+            qi, kj = pos(i), pos(j)
+            a, b, c = block_backward_share(q[:, :, qi], k[:, :, kj], v[:, :, kj], g[:, :, qi],
+                                           lse[:, :, qi], dlt[:, :, qi], 0.5, True, qi, kj)
+            dq[:, :, qi] += a
+            dk[:, :, kj] += b
+            dv[:, :, kj] += c
+    for x, y in zip((dq, dk, dv), want):
+        assert np.abs(x - y).max() <= 1e-12
