@@ -29,6 +29,14 @@ Transports:
   * ``HostTransport`` -- send / recv through host memory (a gloo process
     group, or CPU tensors); the exchange is synchronous.
 
+Ulysses (page "AI 推理系列（十一）…", section "Ring 与 Ulysses：同样切序列，通信
+方式不同"): the same token partitions are re-sharded before attention by an
+all-to-all of Q, K, V so that every device holds a share of the heads over
+the whole sequence, attends locally, and a second all-to-all restores the
+sequence layout.  ``ulysses_attention_forward`` / ``_backward`` implement it
+with the library's single-device kernels for the local attention; the head
+count must split evenly over the devices (H_q % P == H_kv % P == 0).
+
 The block arithmetic is a pluggable ``blocks`` object; ``KernelBlocks`` (the
 default) runs the library's CUDA kernels.
 """
@@ -40,7 +48,8 @@ import torch.distributed as dist
 from . import ra
 
 __all__ = ["KernelBlocks", "NcclTransport", "HostTransport", "default_transport",
-           "ring_attention_forward", "ring_attention_backward", "partition_positions"]
+           "ring_attention_forward", "ring_attention_backward", "partition_positions",
+           "ulysses_attention_forward", "ulysses_attention_backward"]
 
 
 class KernelBlocks:
@@ -61,10 +70,21 @@ class KernelBlocks:
         ra.block_backward(q, k, v, dout, lse, delta, q_offset, k_offset, stride, causal, scale,
                           dq_acc, dk_acc, dv_acc)
 
+    def full(self, q, k, v, causal, scale):
+        return ra.ring_forward(q, k, v, 1, causal, scale)
+
+    def full_backward(self, q, k, v, out, lse, dout, causal, scale):
+        return ra.ring_backward(q, k, v, out, lse, dout, 1, causal, scale)
+
 
 class _Done:
     def wait(self):
         return None
+
+
+def _peer(group, r):
+    """Global rank of rank `r` of `group` (point-to-point calls take global ranks)."""
+    return r if group is None else dist.get_global_rank(group, r)
 
 
 class NcclTransport:
@@ -75,6 +95,7 @@ class NcclTransport:
         self.group = group
 
     def exchange(self, send, recv, nxt, prv):
+        nxt, prv = _peer(self.group, nxt), _peer(self.group, prv)
         ops = [dist.P2POp(dist.isend, t, nxt, self.group) for t in send]
         ops += [dist.P2POp(dist.irecv, t, prv, self.group) for t in recv]
         reqs = dist.batch_isend_irecv(ops)
@@ -84,6 +105,10 @@ class NcclTransport:
                 for r in reqs:
                     r.wait()
         return _Handle()
+
+    def all_to_all(self, send, recv):
+        """send[c] goes to rank c, recv[c] comes from rank c (device tensors)."""
+        dist.all_to_all(recv, send, group=self.group)
 
 
 class HostTransport:
@@ -96,6 +121,7 @@ class HostTransport:
 
     def exchange(self, send, recv, nxt, prv):
         me = dist.get_rank(self.group)
+        nxt, prv = _peer(self.group, nxt), _peer(self.group, prv)
         staged = [t.detach().to("cpu") for t in send]
         bufs = [torch.empty(t.shape, dtype=t.dtype) for t in recv]
         # even ranks send first, odd ranks receive first: no cycle of blocking sends
@@ -109,6 +135,24 @@ class HostTransport:
         for b, t in zip(bufs, recv):
             t.copy_(b)
         return _Done()
+
+    def all_to_all(self, send, recv):
+        """send[c] goes to rank c, recv[c] comes from rank c; completes before
+        returning."""
+        me = dist.get_rank(self.group)
+        staged = [t.detach().to("cpu").contiguous() for t in send]
+        bufs = [torch.empty(t.shape, dtype=t.dtype) for t in recv]
+        bufs[me].copy_(staged[me])
+        reqs = []
+        for c in range(len(send)):
+            if c != me:
+                peer = _peer(self.group, c)
+                reqs.append(dist.isend(staged[c], peer, self.group))
+                reqs.append(dist.irecv(bufs[c], peer, self.group))
+        for r in reqs:
+            r.wait()
+        for b, t in zip(bufs, recv):
+            t.copy_(b)
 
 
 def default_transport(group=None):
@@ -194,3 +238,60 @@ def ring_attention_backward(q, k, v, out, lse, dout, causal=True, scale=None, st
             kv, kv_buf = kv_buf, kv
     # after P accumulator hops every rank holds its own dK, dV
     return dq.to(q.dtype), acc[0].to(k.dtype), acc[1].to(v.dtype)
+
+
+def _seq_to_heads(x, P, transport):
+    """[B, H, L, d] sequence partition of every head -> [B, H / P, P * L, d]:
+    this rank's head share over the whole sequence (partitions in rank
+    order)."""
+    B, H, L = x.shape[:3]
+    hp = H // P
+    send = [x[:, c * hp:(c + 1) * hp].contiguous() for c in range(P)]
+    recv = [torch.empty_like(send[0]) for _ in range(P)]
+    transport.all_to_all(send, recv)
+    return torch.cat(recv, dim=2)
+
+
+def _heads_to_seq(y, P, transport):
+    """Inverse of ``_seq_to_heads``: [B, H / P, P * L, ...] -> [B, H, L, ...]."""
+    L = y.shape[2] // P
+    send = [y[:, :, c * L:(c + 1) * L].contiguous() for c in range(P)]
+    recv = [torch.empty_like(send[0]) for _ in range(P)]
+    transport.all_to_all(send, recv)
+    return torch.cat(recv, dim=1)
+
+
+def _ulysses_check(q, k, P):
+    if q.shape[1] % P or k.shape[1] % P:
+        raise ValueError(f"Ulysses needs H_q ({q.shape[1]}) and H_kv ({k.shape[1]}) divisible "
+                         f"by the {P} devices")
+
+
+def ulysses_attention_forward(q, k, v, causal=True, scale=None, group=None, transport=None,
+                              blocks=None):
+    """This rank's output (O_i [B, Hq, L, d_v], LSE_i [B, Hq, L]) of exact
+    attention over the whole sequence; rank r holds the contiguous tokens
+    [r L, (r + 1) L) of every head on entry and on return."""
+    P = dist.get_world_size(group)
+    transport = transport or default_transport(group)
+    blocks = blocks or KernelBlocks()
+    _ulysses_check(q, k, P)
+    scale = q.shape[-1] ** -0.5 if scale is None else scale
+    qh, kh, vh = (_seq_to_heads(x, P, transport) for x in (q, k, v))
+    o, lse = blocks.full(qh, kh, vh, causal, scale)
+    return (_heads_to_seq(o, P, transport),
+            _heads_to_seq(lse.unsqueeze(-1), P, transport)[..., 0].contiguous())
+
+
+def ulysses_attention_backward(q, k, v, out, lse, dout, causal=True, scale=None, group=None,
+                               transport=None, blocks=None):
+    """This rank's gradients (dQ_i, dK_i, dV_i) of ``ulysses_attention_forward``."""
+    P = dist.get_world_size(group)
+    transport = transport or default_transport(group)
+    blocks = blocks or KernelBlocks()
+    _ulysses_check(q, k, P)
+    scale = q.shape[-1] ** -0.5 if scale is None else scale
+    qh, kh, vh, oh, gh = (_seq_to_heads(x, P, transport) for x in (q, k, v, out, dout))
+    lh = _seq_to_heads(lse.unsqueeze(-1), P, transport)[..., 0].contiguous()
+    dq, dk, dv = blocks.full_backward(qh, kh, vh, oh, lh, gh, causal, scale)
+    return tuple(_heads_to_seq(x, P, transport) for x in (dq, dk, dv))

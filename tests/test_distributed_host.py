@@ -1,9 +1,11 @@
-"""CPU tests of the multi-device ring (ring_context_parallelism_ra_b200/
-distributed.py) over gloo with world sizes 2 and 3.  The block arithmetic is
+"""CPU tests of the multi-device ring and of the Ulysses all-to-all variant
+(ring_context_parallelism_ra_b200/distributed.py) over gloo with world sizes
+2 and 3.  The block arithmetic is
 supplied by the fp64 oracle (a test-only ``blocks`` object), so these tests
 check the ring's own logic: the exchange schedule, the causal skip of a
 contiguous split, the striped positions, the final merge, and the routing of
-the travelling gradient accumulators back to their owners.  Each rank's
+the travelling gradient accumulators back to their owners, and Ulysses' head
+re-shard and its inverse.  Each rank's
 result is compared with the oracle's whole-sequence attention and gradients."""
 import datetime
 import os
@@ -50,6 +52,16 @@ class OracleBlocks:
     def delta(self, out, dout):
         from oracle.backward import row_delta
         return torch.from_numpy(row_delta(out, dout))
+
+    def full(self, q, k, v, causal, scale):
+        from oracle.attention import attention
+        oo, ll = attention(q, k, v, scale, causal)
+        return torch.from_numpy(oo).to(q.dtype), torch.from_numpy(ll).float()
+
+    def full_backward(self, q, k, v, out, lse, dout, causal, scale):
+        from oracle.backward import attention_backward
+        return tuple(torch.from_numpy(x).to(q.dtype)
+                     for x in attention_backward(q, k, v, dout, scale, causal))
 
     def backward(self, q, k, v, dout, lse, delta, q_offset, k_offset, stride, causal, scale,
                  dq_acc, dk_acc, dv_acc):
@@ -111,6 +123,64 @@ def test_ring_over_gloo_matches_whole_sequence(world, striped, causal):
     port = _free_port()
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, striped, causal, errq))
              for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    errs = []
+    while not errq.empty():
+        errs.append(errq.get())
+    assert not errs, errs
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+
+
+def _ulysses_main(rank, world, port, errq):
+    import torch.distributed as dist
+
+    from oracle.attention import attention
+    from oracle.backward import attention_backward
+    from ring_context_parallelism_ra_b200.distributed import (HostTransport,
+                                                              ulysses_attention_backward,
+                                                              ulysses_attention_forward)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, L, d, dv = 2, 7, 5, 4
+        Hq, Hkv = 2 * world, world
+        n = L * world
+        rng = np.random.default_rng(2000 + world)
+        q = torch.from_numpy(rng.standard_normal((B, Hq, n, d)))
+        k = torch.from_numpy(rng.standard_normal((B, Hkv, n, d)))
+        v = torch.from_numpy(rng.standard_normal((B, Hkv, n, dv)))
+        g = torch.from_numpy(rng.standard_normal((B, Hq, n, dv)))
+        rows = np.arange(rank * L, (rank + 1) * L)
+        part = lambda x: x[:, :, rows].contiguous()  # noqa: E731
+        tr, blocks = HostTransport(), OracleBlocks()
+        out, lse = ulysses_attention_forward(part(q), part(k), part(v), True, 0.4,
+                                             transport=tr, blocks=blocks)
+        want_o, want_l = attention(q, k, v, 0.4, True)
+        assert out.shape == (B, Hq, L, dv) and lse.shape == (B, Hq, L)
+        assert np.abs(out.numpy() - want_o[:, :, rows]).max() <= 1e-6
+        assert np.abs(lse.numpy() - want_l[:, :, rows]).max() <= 1e-5
+        grads = ulysses_attention_backward(part(q), part(k), part(v), out, lse, part(g), True, 0.4,
+                                           transport=tr, blocks=blocks)
+        want = attention_backward(q, k, v, g, 0.4, True)
+        for got, w in zip(grads, want):
+            assert np.abs(got.numpy() - w[:, :, rows]).max() <= 1e-9
+    except Exception:
+        errq.put((rank, traceback.format_exc()))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ulysses_over_gloo_matches_whole_sequence(world):
+    ctx = mp.get_context("spawn")
+    errq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ulysses_main, args=(r, world, port, errq)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:

@@ -1,4 +1,5 @@
-"""The multi-device ring (distributed.py) with the library's kernels: two ranks
+"""The multi-device ring and the Ulysses variant (distributed.py) with the
+library's kernels: two ranks
 as two processes on one GPU, exchanging K/V and the travelling gradient
 accumulators through host memory (gloo, HostTransport).  No kernel waits on
 another rank's kernel; only the hosts exchange data.  Each rank's output and
@@ -28,7 +29,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, striped, errq):
+def _rank_main(rank, world, port, mode, errq):
     import torch.distributed as dist
 
     from oracle.attention import attention
@@ -36,7 +37,9 @@ def _rank_main(rank, world, port, striped, errq):
     from ring_context_parallelism_ra_b200 import ra
     from ring_context_parallelism_ra_b200.distributed import (HostTransport,
                                                               ring_attention_backward,
-                                                              ring_attention_forward)
+                                                              ring_attention_forward,
+                                                              ulysses_attention_backward,
+                                                              ulysses_attention_forward)
     from ring_context_parallelism_ra_b200.workloads import make_dout, make_qkv
     from tests.parity_util import check_grad, check_lse, check_out
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -48,18 +51,28 @@ def _rank_main(rank, world, port, striped, errq):
         n = L * world
         q, k, v = make_qkv(B, Hq, Hkv, n, n, d, d, torch.bfloat16, seed=61 + world)
         g = make_dout(B, Hq, n, d, torch.bfloat16, seed=61 + world)
+        striped = mode == "striped"
         rows = (np.arange(rank, n, world) if striped
                 else np.arange(rank * L, (rank + 1) * L))
         part = lambda x: x[:, :, rows].contiguous().to("cuda")  # noqa: E731
         scale = 1 / math.sqrt(d)
         tr = HostTransport()
-        out, lse = ring_attention_forward(part(q), part(k), part(v), True, scale, striped,
-                                          transport=tr)
+        if mode == "ulysses":
+            fwd = lambda: ulysses_attention_forward(part(q), part(k), part(v), True, scale,  # noqa: E731
+                                                    transport=tr)
+            bwd = lambda o, l: ulysses_attention_backward(part(q), part(k), part(v), o, l,  # noqa: E731
+                                                          part(g), True, scale, transport=tr)
+        else:
+            fwd = lambda: ring_attention_forward(part(q), part(k), part(v), True, scale,  # noqa: E731
+                                                 striped, transport=tr)
+            bwd = lambda o, l: ring_attention_backward(part(q), part(k), part(v), o, l,  # noqa: E731
+                                                       part(g), True, scale, striped,
+                                                       transport=tr)
+        out, lse = fwd()
         want_o, want_l = attention(q, k, v, scale, True)
         check_out(out, want_o[:, :, rows], "bf16")
         check_lse(lse, want_l[:, :, rows])
-        dq, dk, dv = ring_attention_backward(part(q), part(k), part(v), out, lse, part(g), True,
-                                             scale, striped, transport=tr)
+        dq, dk, dv = bwd(out, lse)
         wq, wk, wv = attention_backward(q, k, v, g, scale, True)
         check_grad(dq, wq[:, :, rows], "bf16", "dQ")
         check_grad(dk, wk[:, :, rows], "bf16", "dK")
@@ -72,13 +85,13 @@ def _rank_main(rank, world, port, striped, errq):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("striped", [False, True])
-def test_two_rank_ring_on_one_gpu_matches_oracle(striped):
+@pytest.mark.parametrize("mode", ["contiguous", "striped", "ulysses"])
+def test_two_rank_ring_on_one_gpu_matches_oracle(mode):
     assert torch.cuda.is_available()
     ctx = mp.get_context("spawn")
     errq = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, striped, errq)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, mode, errq)) for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
