@@ -260,3 +260,23 @@ def test_library_rejects_host_pointer_shapes():
     with pytest.raises(ra.RAError) as e:
         ra.ring_forward(q, k, k, 1, True)
     assert e.value.status == ra.RA_ERR_INVALID
+
+
+def test_host_pipeline_equals_direct_calls():
+    # The overlapped host pipeline returns, for every batch, exactly what a
+    # direct ring_forward on the same inputs returns (same kernel).
+    from ring_context_parallelism_ra_b200.host_pipeline import RingForwardPipeline
+    shape = (1, 4, 2, 640, 640, 128, 128)
+    batches = [make_qkv(*shape, torch.bfloat16, seed=300 + i) for i in range(5)]
+    pipe = RingForwardPipeline(batches[0][0].shape, batches[0][1].shape, batches[0][2].shape,
+                               torch.bfloat16, 4, True)
+    pinned = [tuple(x.pin_memory() for x in b) for b in batches]
+    for i, (q, k, v) in enumerate(pinned):
+        slot = pipe.submit(q, k, v)
+        if i >= 1:  # results of the previous batch while this one is in flight
+            o_prev, l_prev = pipe.wait((slot - 1) % pipe.depth)
+            want_o, want_l = ra.ring_forward(*(x.to(DEV) for x in batches[i - 1]), 4, True)
+            assert torch.equal(o_prev, want_o.cpu()) and torch.equal(l_prev, want_l.cpu())
+    o_last, l_last = pipe.wait((len(batches) - 1) % pipe.depth)
+    want_o, want_l = ra.ring_forward(*(x.to(DEV) for x in batches[-1]), 4, True)
+    assert torch.equal(o_last, want_o.cpu()) and torch.equal(l_last, want_l.cpu())
