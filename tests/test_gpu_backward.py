@@ -219,3 +219,39 @@ def test_backward_sampled_at_8k_mha_workload():
     assert (np.abs(dk64.sum(axis=2)) <= bar(dk64)).all()
     want_sv = to64(g).reshape(wl.B, wl.Hkv, -1, wl.n, wl.d_v).sum(axis=(2, 3))
     assert (np.abs(dv64.sum(axis=2) - want_sv) <= bar(dv64)).all()
+
+
+@pytest.mark.parametrize("dt", [BF, F32])
+def test_block_backward_rows_without_keys_and_noncausal(dt):
+    # Keys placed after every query of the first rows: those rows see no key
+    # (LSE -inf) and get no gradient; a non-causal block with a ragged tail.
+    B, Hq, Hkv, nq, nk, d = 1, 8, 1, 200, 130, 64
+    q, k, v = make_qkv(B, Hq, Hkv, nq, nk, d, d, dt, seed=81)
+    g = make_dout(B, Hq, nq, d, dt, seed=81)
+    scale = 1 / math.sqrt(d)
+    for causal, ko in ((True, 60), (False, 0)):
+        o, l = oracle_attention(q, k, v, scale, causal, q_offset=0, k_offset=ko)
+        lse = torch.tensor(l, dtype=torch.float32, device=DEV)
+        delta = torch.tensor(row_delta(o, g), dtype=torch.float32, device=DEV)
+        dq, dk, dv = ra.block_backward(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), lse, delta,
+                                       q_offset=0, k_offset=ko, causal=causal)
+        want = attention_backward(q, k, v, g, scale, causal, q_offset=0, k_offset=ko)
+        kind = _kind(dt)
+        check_grad(dq, want[0], kind, "dQ")
+        check_grad(dk, want[1], kind, "dK")
+        check_grad(dv, want[2], kind, "dV")
+        if causal:
+            assert (dq[:, :, :ko] == 0).all()   # rows 0..59 see no key
+
+
+def test_ring_backward_gqa_8_to_1_ragged():
+    B, Hq, Hkv, n, d, P = 1, 8, 1, 700, 128, 7
+    q, k, v = make_qkv(B, Hq, Hkv, n, n, d, d, BF, seed=91)
+    g = make_dout(B, Hq, n, d, BF, seed=91)
+    qd, kd, vd, gd = (x.to(DEV) for x in (q, k, v, g))
+    out, lse = ra.ring_forward(qd, kd, vd, P, True)
+    dq, dk, dv = ra.ring_backward(qd, kd, vd, out, lse, gd, P, True)
+    want = attention_backward(q, k, v, g, 1 / math.sqrt(d), True)
+    check_grad(dq, want[0], "bf16", "dQ")
+    check_grad(dk, want[1], "bf16", "dK")
+    check_grad(dv, want[2], "bf16", "dV")
