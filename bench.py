@@ -21,6 +21,7 @@ from __future__ import annotations
 import argparse
 import dataclasses
 import hashlib
+import re
 import json
 import math
 import os
@@ -55,11 +56,20 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(text):
+    """Source text without comments and with whitespace collapsed, so that a
+    hash of it changes with the code and not with its commentary."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_sha(files):
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "ring_context_parallelism_ra_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "ring_context_parallelism_ra_b200", "csrc", f),
+                  encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

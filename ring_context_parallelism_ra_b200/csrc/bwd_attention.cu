@@ -35,9 +35,11 @@
 // dP^T), dV [256,256+DV), dK [256+DV,256+DV+DQK).
 // Products per visit v and their issuers: A issues dV(v) then S^T(v+1), B
 // issues dK(v), C issues dQ(v) then dP^T(v+1).  MMAs of one thread execute
-// in issue order, so S^T(v+1) overwrites P^T(v) only after dV(v) has read it
-// and dP^T(v+1) overwrites dQ(v) only after it was read out; the compute
-// warps form P^T(v+1) while the tensor cores run dK(v) and dQ(v).
+// in issue order, so S^T(v+1) overwrites P^T(v) only after dV(v) has read
+// it; dP^T(v+1) waits until the compute warps have read dQ(v) out; the
+// compute warps form P^T(v+1) while the tensor cores run dK(v) and dQ(v).
+// Where the products of two issuers meet (the stage of Q / dO, the K / V
+// tile, the finished dK / dV) the barrier takes one commit from each.
 #include <cuda.h>
 
 #include "block_class.cuh"

@@ -99,3 +99,18 @@ def test_flop_and_byte_counts_match_oracle_formulas():
     wl = workload(4)
     assert decode_kv_bytes(wl) == wl.B * kv_cache_bytes(1, wl.Hkv, wl.d_qk, wl.n, 2)
     assert decode_kv_bytes(wl) == 17179869184
+
+
+def test_kernel_source_hash_follows_code_not_comments():
+    a = "int f(int x) {  // doubles\n  return 2 * x; /* fast */ }\n"
+    b = "/* header */ int f(int x) {\n    return 2 * x;\n}  // end\n"
+    c = "int f(int x) { return 3 * x; }"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+
+
+def test_committed_traffic_matches_current_kernel_sources():
+    # profiles/traffic.json holds DRAM bytes captured on the kernels' current
+    # code; the bench reports them only while the code is unchanged
+    assert bench.load_traffic("ring_forward:causal_mha_b1_h8_n8192_d128_P4", bench.TC_FILES)
+    assert bench.load_traffic("ring_backward:causal_mha_b1_h8_n8192_d128_P4", bench.BWD_FILES)
