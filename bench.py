@@ -290,6 +290,7 @@ def run_ours(args, world, rank):
 
     decode = None if args.skip_decode else run_decode_leg(args, world, rank, peaks, peaks_kind)
     striped = None if args.skip_striped else run_striped_leg(args, world, rank, workload(3), peaks)
+    merge = None if args.skip_merge else run_merge_leg(args, world, rank, peaks, peaks_kind)
     backward = None
     if not args.skip_backward and wl.dtype == "bf16":
         backward = [run_backward_leg(args, world, rank, w, peaks, peaks_kind)
@@ -316,7 +317,57 @@ def run_ours(args, world, rank):
         line["striped"] = striped
     if backward is not None:
         line["backward"] = backward
+    if merge is not None:
+        line["merge"] = merge
     return line
+
+
+def run_merge_leg(args, world, rank, peaks, peaks_kind):
+    """ra_lse_merge alone on the partials one query partition of a ring
+    collects (P normalised fp32 partials and their LSE): the 8K MHA shape
+    (P = 4 partials of [1, 8, 2048, 128]) and the 128K GQA shape (P = 8
+    partials of [1, 32, 16384, 128], 2 GiB).  GB/s over the bytes read and
+    written."""
+    dev = torch.device("cuda")
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    stream = torch.cuda.current_stream()
+    res = []
+    for key in (2, 3):
+        wl = workload(key)
+        L = wl.n // wl.P
+        g = torch.Generator(device=dev).manual_seed(wl.seed + 7 + 1000 * rank)
+        o = torch.randn((wl.P, wl.B, wl.Hq, L, wl.d_v), device=dev, generator=g)
+        l = torch.randn((wl.P, wl.B, wl.Hq, L), device=dev, generator=g) * 3
+        out = torch.empty((wl.B, wl.Hq, L, wl.d_v), device=dev, dtype=wl.torch_dtype)
+        lse = torch.empty((wl.B, wl.Hq, L), device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            ra.lse_merge(o, l, wl.torch_dtype, out, lse)
+        steps = max(3, min(args.steps, 10))
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ra.lse_merge(o, l, wl.torch_dtype, out, lse)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        assert ra.get_status() == ra.RA_OK
+        ms = max_over_ranks(statistics.mean(ts), world)
+        nbytes = (o.numel() + l.numel()) * 4 + out.numel() * out.element_size() + lse.numel() * 4
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res.append({"shape": f"{wl.name}: P={wl.P} partials of [{wl.B}, {wl.Hq}, {L}, {wl.d_v}]",
+                    "value": round(world * gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
+                    "bytes_per_step": nbytes,
+                    "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                                 "unit": "GB/s", "frac": round(gbs / peak, 4),
+                                 "peak_kind": f"{peaks_kind} HBM copy",
+                                 "kernel": "lse_merge_kernel"}})
+        del o, l, out, lse, flush
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_backward_leg(args, world, rank, wl, peaks, peaks_kind):
@@ -541,6 +592,7 @@ def main():
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-striped", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
+    ap.add_argument("--skip-merge", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:
