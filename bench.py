@@ -364,7 +364,7 @@ def run_merge_leg(args, world, rank, peaks, peaks_kind):
                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
                                  "unit": "GB/s", "frac": round(gbs / peak, 4),
                                  "peak_kind": f"{peaks_kind} HBM copy",
-                                 "kernel": "lse_merge_kernel"}})
+                                 "kernel": "lse_merge_few_kernel" if wl.P <= 4 else "lse_merge_kernel"}})
         del o, l, out, lse, flush
         torch.cuda.empty_cache()
     return res

@@ -76,6 +76,62 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
   }
 }
 
+// The same merge with at most MAXP partials: every LSE and O load of a row is
+// issued before any arithmetic, so a row costs one trip to memory instead of
+// two (the LSE maxima first, then the weighted sum).
+template <typename OutT, int MAXP>
+__global__ void __launch_bounds__(256) lse_merge_few_kernel(const float* __restrict__ o_parts,
+                                                            const float* __restrict__ lse_parts,
+                                                            int P, long long rows, int d_v,
+                                                            OutT* __restrict__ out,
+                                                            float* __restrict__ lse_out) {
+  const int lanes_per_row = d_v >> 2;
+  const int rows_per_warp = 32 / lanes_per_row;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / lanes_per_row;
+  const int col = (lane % lanes_per_row) * 4;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const long long part_stride = rows * d_v;
+  for (long long r = warp * rows_per_warp + sub; r < rows; r += n_warps * rows_per_warp) {
+    float l[MAXP];
+    float4 o[MAXP];
+    const float* src = o_parts + r * d_v + col;
+#pragma unroll
+    for (int p = 0; p < MAXP; ++p) {
+      if (p < P) {
+        l[p] = __ldg(lse_parts + p * rows + r);
+        o[p] = __ldcs(reinterpret_cast<const float4*>(src + p * part_stride));
+      }
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int p = 0; p < MAXP; ++p)
+      if (p < P) m = fmaxf(m, l[p]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float w_sum = 0.f;
+    if (m != -INFINITY) {
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        if (p < P) {
+          const float w = (l[p] == -INFINITY) ? 0.f : expf(l[p] - m);
+          w_sum += w;
+          acc.x = fmaf(w, o[p].x, acc.x);
+          acc.y = fmaf(w, o[p].y, acc.y);
+          acc.z = fmaf(w, o[p].z, acc.z);
+          acc.w = fmaf(w, o[p].w, acc.w);
+        }
+      }
+      const float inv = 1.f / w_sum;
+      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+    }
+    store4<OutT>(out + r * d_v + col, acc);
+    if (lse_out != nullptr && col == 0) {
+      lse_out[r] = (m == -INFINITY) ? -INFINITY : m + logf(w_sum);
+    }
+  }
+}
+
 // Few rows, many partials (the chunk partials of one decode shard): the
 // row-per-warp kernel above would leave the GPU nearly idle and walk P
 // partials serially.  Here eight warps share each row group, warp w taking
@@ -173,7 +229,16 @@ int launch_lse_merge(const float* o_parts, const float* lse_parts, int P, long l
     long long cap = static_cast<long long>(num_sms) * 8;   // 8 resident CTAs / SM
     int grid = static_cast<int>(want < cap ? want : cap);
     if (grid < 1) grid = 1;
-    if (out_dtype == RA_F32) {
+    // Up to four partials fit in registers at 48 per thread; more would cut the
+    // resident warps (8 partials: 70 registers, 24 warps per SM instead of 64)
+    // and lose more than the single round trip gains, so those loop.
+    if (P <= 4 && out_dtype == RA_F32) {
+      lse_merge_few_kernel<float, 4><<<grid, threads, 0, stream>>>(
+          o_parts, lse_parts, P, rows, d_v, static_cast<float*>(out), lse);
+    } else if (P <= 4) {
+      lse_merge_few_kernel<__nv_bfloat16, 4><<<grid, threads, 0, stream>>>(
+          o_parts, lse_parts, P, rows, d_v, static_cast<__nv_bfloat16*>(out), lse);
+    } else if (out_dtype == RA_F32) {
       lse_merge_kernel<float><<<grid, threads, 0, stream>>>(o_parts, lse_parts, P, rows, d_v,
                                                             static_cast<float*>(out), lse);
     } else {

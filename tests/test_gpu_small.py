@@ -53,6 +53,8 @@ def test_lse_merge_matches_oracle(P, dv, out_dtype):
 
 
 @pytest.mark.parametrize("P,B,H,n,dv", [(8, 1, 8, 4096, 128),    # many rows: one warp per row
+                                        (4, 1, 8, 2048, 128),    # P <= 4: all loads issued at once
+                                        (24, 1, 2, 2048, 128),   # P > 16, many rows: looped row kernel
                                         (12, 1, 3, 37, 64),      # few rows, odd count: split-P
                                         (64, 4, 64, 1, 128),     # decode chunk partials
                                         (9, 2, 2, 5, 32)])
