@@ -474,6 +474,8 @@ def run_striped_leg(args, world, rank, wl, peaks):
 
     ms_striped = timed(lambda: ra.ring_forward_striped(qs, ks, vs, P, wl.causal, wl.scale, out, lse))
     ms_contig = timed(lambda: ra.ring_forward(q, k, v, P, wl.causal, wl.scale, out, lse))
+    # T(cp = 1): the whole sequence as one partition on this one device
+    ms_one = timed(lambda: ra.ring_forward(q, k, v, 1, wl.causal, wl.scale, out, lse))
     parts = {}
     for name, (qq, kk, vv) in (("contiguous", (q, k, v)), ("striped", (qs, ks, vs))):
         qi = [qq[:, :, i * L:(i + 1) * L].contiguous() for i in range(P)]
@@ -503,6 +505,11 @@ def run_striped_leg(args, world, rank, wl, peaks):
            "slowest_device_ms": {k: round(max(v), 4) for k, v in parts.items()},
            "ring_speedup_striped_over_contiguous":
                round(max(parts["contiguous"]) / max(parts["striped"]), 3),
+           # scaling efficiency eta(cp) = T(cp = 1) / (cp T(cp)), T(cp) = the
+           # slowest emulated device (the exchange, hidden under the blocks on
+           # NVLink, and the final merge are not in it)
+           "t_cp1_ms": round(ms_one, 4),
+           "eta_cp": {k: round(ms_one / (P * max(v)), 4) for k, v in parts.items()},
            "note": "block partials per emulated device, one device at a time on this GPU"}
     del q, k, v, qs, ks, vs, out, lse, flush
     torch.cuda.empty_cache()

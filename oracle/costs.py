@@ -7,7 +7,8 @@ and that these reproduce the pages' worked numbers.
 from __future__ import annotations
 
 __all__ = ["kv_cache_bytes", "decode_latency_lower_bound_s", "prefill_flops",
-           "backward_flops", "pass_kv_bytes_per_chip", "kv_bytes_per_chip", "mla_ckv_bytes"]
+           "backward_flops", "pass_kv_bytes_per_chip", "kv_bytes_per_chip", "mla_ckv_bytes",
+           "prefill_compute_time_s", "prefill_time_s", "scaling_efficiency"]
 
 
 def kv_cache_bytes(L, h_kv, d_h, n, b):
@@ -57,3 +58,24 @@ def mla_ckv_bytes(kv_lora_rank, rope_dim, bytes_per_value):
     decoupled RoPE key), page "上下文并行 (CP) 收益评估实验设计", table of fixed
     parameters (c_kv for DeepSeek-V3 in BF16)."""
     return (kv_lora_rank + rope_dim) * bytes_per_value
+
+
+def prefill_compute_time_s(B, S, d_qk, d_v, cp, R):
+    """Page "上下文并行 (CP) 收益评估实验设计", Eq. (cpeval-comp): each of the cp
+    chips computes 2 B S^2 (D_qk + D_v) / cp FLOPs at an effective rate of R
+    FLOP/s, so T_comp = 2 B S^2 (D_qk + D_v) / (cp R) (one head, full square,
+    as the page writes it)."""
+    return 2 * B * S * S * (d_qk + d_v) / (cp * R)
+
+
+def prefill_time_s(t_comp, t_passkv):
+    """Same page, Eq. (cpeval-prefill): with the ring exchange overlapped with
+    the block computation the slower of the two is the critical path,
+    T_prefill = max(T_comp, T_passkv)."""
+    return max(t_comp, t_passkv)
+
+
+def scaling_efficiency(t_1, t_cp, cp):
+    """Same page, terms table ("scaling 效率"): eta(cp) = T(cp = 1) / (cp T(cp)),
+    1 for a linear speed-up."""
+    return t_1 / (cp * t_cp)

@@ -37,6 +37,15 @@ sequence layout.  ``ulysses_attention_forward`` / ``_backward`` implement it
 with the library's single-device kernels for the local attention; the head
 count must split evenly over the devices (H_q % P == H_kv % P == 0).
 
+Pass-Q decode (page "上下文并行 (CP) 收益评估实验设计", decode section and the
+pass-KV / pass-Q term): the KV cache is split by token range, one shard per
+device; the single query token of each sequence goes to every device, each
+device computes the normalised partial attention of the query over its own
+shard, and the partials are reduced.  ``pass_q_decode`` sends the query from
+one rank, gathers every rank's (O_p, LSE_p) in one collective, and merges
+them with the log-sum-exp rule on every rank, so all ranks return the same
+result.
+
 The block arithmetic is a pluggable ``blocks`` object; ``KernelBlocks`` (the
 default) runs the library's CUDA kernels.
 """
@@ -49,7 +58,7 @@ from . import ra
 
 __all__ = ["KernelBlocks", "NcclTransport", "HostTransport", "default_transport",
            "ring_attention_forward", "ring_attention_backward", "partition_positions",
-           "ulysses_attention_forward", "ulysses_attention_backward"]
+           "ulysses_attention_forward", "ulysses_attention_backward", "pass_q_decode"]
 
 
 class KernelBlocks:
@@ -75,6 +84,12 @@ class KernelBlocks:
 
     def full_backward(self, q, k, v, out, lse, dout, causal, scale):
         return ra.ring_backward(q, k, v, out, lse, dout, 1, causal, scale)
+
+    def decode_partial(self, q, k, v, scale, o_part, lse_part):
+        ra.decode_partial(q, k, v, scale=scale, o_part=o_part, lse_part=lse_part)
+
+    def decode_merge(self, o_parts, lse_parts, out_dtype):
+        return ra.decode_merge(o_parts, lse_parts, out_dtype)
 
 
 class _Done:
@@ -109,6 +124,14 @@ class NcclTransport:
     def all_to_all(self, send, recv):
         """send[c] goes to rank c, recv[c] comes from rank c (device tensors)."""
         dist.all_to_all(recv, send, group=self.group)
+
+    def broadcast(self, t, src):
+        """Overwrite `t` on every rank with rank `src`'s `t`."""
+        dist.broadcast(t, _peer(self.group, src), group=self.group)
+
+    def all_gather(self, out, inp):
+        """out[c] = rank c's `inp` (out: [P, *inp.shape], contiguous)."""
+        dist.all_gather_into_tensor(out, inp, group=self.group)
 
 
 class HostTransport:
@@ -153,6 +176,20 @@ class HostTransport:
             r.wait()
         for b, t in zip(bufs, recv):
             t.copy_(b)
+
+    def broadcast(self, t, src):
+        """Overwrite `t` on every rank with rank `src`'s `t`; completes before
+        returning."""
+        staged = t.detach().to("cpu").contiguous()
+        dist.broadcast(staged, _peer(self.group, src), group=self.group)
+        t.copy_(staged)
+
+    def all_gather(self, out, inp):
+        """out[c] = rank c's `inp`; completes before returning."""
+        staged = inp.detach().to("cpu").contiguous()
+        bufs = [torch.empty(staged.shape, dtype=staged.dtype) for _ in range(out.shape[0])]
+        dist.all_gather(bufs, staged, group=self.group)
+        out.copy_(torch.stack(bufs))
 
 
 def default_transport(group=None):
@@ -295,3 +332,47 @@ def ulysses_attention_backward(q, k, v, out, lse, dout, causal=True, scale=None,
     lh = _seq_to_heads(lse.unsqueeze(-1), P, transport)[..., 0].contiguous()
     dq, dk, dv = blocks.full_backward(qh, kh, vh, oh, lh, gh, causal, scale)
     return tuple(_heads_to_seq(x, P, transport) for x in (dq, dk, dv))
+
+
+def pass_q_decode(q, k_shard, v_shard, scale=None, src=0, group=None, transport=None,
+                  blocks=None):
+    """Decode attention of one query token per sequence over a KV cache split
+    by token range across the ranks of `group`.
+
+    q        : [B, Hq, 1, d_qk]; rank `src`'s copy is sent to every rank
+               (``src=None``: every rank already holds the same q).
+    k_shard,
+    v_shard  : [B, Hkv, S_r, d] -- this rank's tokens of the cache.  The
+               shards need not be equal; an empty shard (S_r = 0) contributes
+               nothing.  Which tokens a rank holds does not matter: decode
+               has no mask, and the merge does not depend on the order.
+    Returns (O [B, Hq, d_v] in q's dtype, LSE fp32 [B, Hq]), the same on
+    every rank.
+
+    One gather moves each rank's O_p and LSE_p together: both are written
+    into one fp32 slot of B * Hq * (d_v + 1) values, the slots of all ranks
+    are gathered, and the stacked partials are taken out of them for the
+    merge."""
+    P = dist.get_world_size(group)
+    transport = transport or default_transport(group)
+    blocks = blocks or KernelBlocks()
+    B, Hq, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence")
+    if src is not None:
+        transport.broadcast(q, src)
+    dv = v_shard.shape[-1]
+    n_o, n_l = B * Hq * dv, B * Hq
+    scale = d ** -0.5 if scale is None else scale
+    gathered = torch.empty((P, n_o + n_l), device=q.device, dtype=torch.float32)
+    slot = torch.empty((n_o + n_l,), device=q.device, dtype=torch.float32)
+    o_p, l_p = slot[:n_o].view(B, Hq, dv), slot[n_o:].view(B, Hq)
+    if k_shard.shape[2] > 0:
+        blocks.decode_partial(q, k_shard, v_shard, scale, o_p, l_p)
+    else:  # no tokens here: the empty partial (weight zero in the merge)
+        o_p.zero_()
+        l_p.fill_(float("-inf"))
+    transport.all_gather(gathered, slot)
+    o_parts = gathered[:, :n_o].reshape(P, B, Hq, dv)
+    l_parts = gathered[:, n_o:].reshape(P, B, Hq)
+    return blocks.decode_merge(o_parts, l_parts, q.dtype)

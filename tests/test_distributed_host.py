@@ -2,10 +2,11 @@
 (ring_context_parallelism_ra_b200/distributed.py) over gloo with world sizes
 2 and 3.  The block arithmetic is
 supplied by the fp64 oracle (a test-only ``blocks`` object), so these tests
-check the ring's own logic: the exchange schedule, the causal skip of a
+check the ring's own logic: the exchange schedule and its pass-KV bytes, the causal skip of a
 contiguous split, the striped positions, the final merge, and the routing of
 the travelling gradient accumulators back to their owners, and Ulysses' head
-re-shard and its inverse.  Each rank's
+re-shard and its inverse, and pass-Q decode (query sent from one rank,
+partials gathered and merged on every rank).  Each rank's
 result is compared with the oracle's whole-sequence attention and gradients."""
 import datetime
 import os
@@ -63,6 +64,15 @@ class OracleBlocks:
         return tuple(torch.from_numpy(x).to(q.dtype)
                      for x in attention_backward(q, k, v, dout, scale, causal))
 
+    def decode_partial(self, q, k, v, scale, o_part, lse_part):
+        from oracle.attention import attention
+        oo, ll = attention(q, k, v, scale, False)
+        o_part.copy_(torch.from_numpy(oo[:, :, 0]))
+        lse_part.copy_(torch.from_numpy(ll[:, :, 0]))
+
+    def decode_merge(self, o_parts, lse_parts, out_dtype):
+        return self.merge(o_parts, lse_parts, out_dtype)
+
     def backward(self, q, k, v, dout, lse, delta, q_offset, k_offset, stride, causal, scale,
                  dq_acc, dk_acc, dv_acc):
         from oracle.backward import block_backward_share
@@ -74,11 +84,24 @@ class OracleBlocks:
         dv_acc += torch.from_numpy(c).to(dv_acc.dtype)
 
 
+def _counting(base):
+    """Wrap a transport so that it counts the bytes this rank sends in ring
+    exchanges."""
+    class Counting(type(base)):
+        sent = 0
+
+        def exchange(self, send, recv, nxt, prv):
+            Counting.sent += sum(t.numel() * t.element_size() for t in send)
+            return super().exchange(send, recv, nxt, prv)
+    return Counting(base.group)
+
+
 def _rank_main(rank, world, port, striped, causal, errq):
     import torch.distributed as dist
 
     from oracle.attention import attention
     from oracle.backward import attention_backward
+    from oracle.costs import pass_kv_bytes_per_chip
     from ring_context_parallelism_ra_b200.distributed import (HostTransport,
                                                               ring_attention_backward,
                                                               ring_attention_forward)
@@ -97,9 +120,13 @@ def _rank_main(rank, world, port, striped, causal, errq):
                 else np.arange(rank * L, (rank + 1) * L))
         part = lambda x: x[:, :, rows].contiguous()  # noqa: E731
         scale = 0.4
-        tr, blocks = HostTransport(), OracleBlocks()
+        tr, blocks = _counting(HostTransport()), OracleBlocks()
         out, lse = ring_attention_forward(part(q), part(k), part(v), causal, scale, striped,
                                           transport=tr, blocks=blocks)
+        # pass-KV traffic of the forward: (cp - 1) / cp * S * c_kv bytes per
+        # rank, c_kv = the K and V bytes of one token over batch and heads
+        c_kv = B * Hkv * (d + dv) * q.element_size()
+        assert type(tr).sent == pass_kv_bytes_per_chip(world, n, c_kv)
         want_o, want_l = attention(q, k, v, scale, causal)
         assert np.abs(out.numpy() - want_o[:, :, rows]).max() <= 1e-6
         assert np.abs(lse.numpy() - want_l[:, :, rows]).max() <= 1e-5
@@ -181,6 +208,58 @@ def test_ulysses_over_gloo_matches_whole_sequence(world):
     errq = ctx.Queue()
     port = _free_port()
     procs = [ctx.Process(target=_ulysses_main, args=(r, world, port, errq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    errs = []
+    while not errq.empty():
+        errs.append(errq.get())
+    assert not errs, errs
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+
+
+def _decode_main(rank, world, port, sizes, errq):
+    import torch.distributed as dist
+
+    from oracle.attention import attention
+    from ring_context_parallelism_ra_b200.distributed import HostTransport, pass_q_decode
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, Hq, Hkv, d, dv = 2, 4, 2, 6, 5
+        n = sum(sizes)
+        rng = np.random.default_rng(3000 + world)
+        q = torch.from_numpy(rng.standard_normal((B, Hq, 1, d)))
+        k = torch.from_numpy(rng.standard_normal((B, Hkv, n, d)))
+        v = torch.from_numpy(rng.standard_normal((B, Hkv, n, dv)))
+        lo = sum(sizes[:rank])
+        shard = slice(lo, lo + sizes[rank])
+        # only rank 1 holds the real query; the others must receive it
+        mine = q.clone() if rank == 1 else torch.full_like(q, 7.0)
+        out, lse = pass_q_decode(mine, k[:, :, shard].contiguous(), v[:, :, shard].contiguous(),
+                                 0.3, src=1, transport=HostTransport(), blocks=OracleBlocks())
+        want_o, want_l = attention(q, k, v, 0.3, False)
+        assert torch.equal(mine, q)
+        assert out.shape == (B, Hq, dv) and lse.shape == (B, Hq)
+        assert np.abs(out.numpy() - want_o[:, :, 0]).max() <= 1e-6
+        assert np.abs(lse.numpy() - want_l[:, :, 0]).max() <= 1e-5
+    except Exception:
+        errq.put((rank, traceback.format_exc()))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("sizes", [(9, 14), (5, 0, 11)])
+def test_pass_q_decode_over_gloo_matches_whole_cache(sizes):
+    world = len(sizes)
+    ctx = mp.get_context("spawn")
+    errq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_decode_main, args=(r, world, port, sizes, errq))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:

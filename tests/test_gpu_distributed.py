@@ -1,5 +1,5 @@
-"""The multi-device ring and the Ulysses variant (distributed.py) with the
-library's kernels: two ranks
+"""The multi-device ring, the Ulysses variant and pass-Q decode
+(distributed.py) with the library's kernels: two ranks
 as two processes on one GPU, exchanging K/V and the travelling gradient
 accumulators through host memory (gloo, HostTransport).  No kernel waits on
 another rank's kernel; only the hosts exchange data.  Each rank's output and
@@ -83,6 +83,57 @@ def _rank_main(rank, world, port, mode, errq):
         raise
     finally:
         dist.destroy_process_group()
+
+
+def _decode_main(rank, world, port, errq):
+    import torch.distributed as dist
+
+    from oracle.attention import attention
+    from ring_context_parallelism_ra_b200 import ra
+    from ring_context_parallelism_ra_b200.distributed import HostTransport, pass_q_decode
+    from ring_context_parallelism_ra_b200.workloads import make_qkv
+    from tests.parity_util import check_lse, check_out
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        B, Hq, Hkv, d = 2, 16, 2, 128
+        sizes = (3000, 5192)                     # ragged shards of an 8192-token cache
+        n = sum(sizes)
+        q, k, v = make_qkv(B, Hq, Hkv, 1, n, d, d, torch.bfloat16, seed=71)
+        lo = sum(sizes[:rank])
+        shard = slice(lo, lo + sizes[rank])
+        mine = (q if rank == 0 else torch.zeros_like(q)).to("cuda")
+        out, lse = pass_q_decode(mine, k[:, :, shard].contiguous().to("cuda"),
+                                 v[:, :, shard].contiguous().to("cuda"), d ** -0.5, src=0,
+                                 transport=HostTransport())
+        want_o, want_l = attention(q, k, v, d ** -0.5, False)
+        check_out(out, want_o[:, :, 0], "bf16")
+        check_lse(lse, want_l[:, :, 0])
+        assert ra.get_status() == ra.RA_OK
+    except Exception:
+        errq.put((rank, traceback.format_exc()))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_pass_q_decode_on_one_gpu_matches_oracle():
+    assert torch.cuda.is_available()
+    ctx = mp.get_context("spawn")
+    errq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_decode_main, args=(r, 2, port, errq)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    errs = []
+    while not errq.empty():
+        errs.append(errq.get())
+    assert not errs, errs
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
 
 
 @pytest.mark.parametrize("mode", ["contiguous", "striped", "ulysses"])

@@ -9,7 +9,8 @@ import pytest
 from oracle.attention import attention
 from oracle.block_class import (FULL, PARTIAL, SKIP, block_class,
                                 block_class_bruteforce, partition_class)
-from oracle.costs import (decode_latency_lower_bound_s, kv_cache_bytes,
+from oracle.costs import (decode_latency_lower_bound_s, kv_cache_bytes, prefill_compute_time_s,
+                          prefill_time_s, scaling_efficiency,
                           mla_ckv_bytes, pass_kv_bytes_per_chip, prefill_flops)
 from oracle.merge import lse_merge
 
@@ -143,3 +144,40 @@ def test_prefill_flops_counts_pairs():
 def test_pass_kv_bytes():
     assert pass_kv_bytes_per_chip(1, 1000, 1152) == 0
     assert pass_kv_bytes_per_chip(8, 1 << 20, 1152) == 7 * (1 << 20) * 1152 / 8
+
+
+def test_prefill_compute_time_is_the_pair_count_split_over_chips():
+    # T_comp * cp * R is the non-causal FLOP count, itself pinned by counting
+    # (query, key) pairs above; the time falls as 1 / cp
+    for B, S, dqk, dv in [(1, 64, 192, 128), (2, 1 << 17, 128, 128)]:
+        for cp in (1, 2, 8):
+            t = prefill_compute_time_s(B, S, dqk, dv, cp, 1e15)
+            assert t * cp * 1e15 == pytest.approx(prefill_flops(B, S, dqk, dv, 1, causal=False))
+        assert prefill_compute_time_s(B, S, dqk, dv, 1, 1e15) == pytest.approx(
+            4 * prefill_compute_time_s(B, S, dqk, dv, 4, 1e15))
+
+
+def test_scaling_efficiency_hidden_and_exposed_regimes():
+    # the page's model: T(cp) = max(T_comp(cp), pass-KV bytes / bandwidth).
+    # While the exchange hides under the computation the speed-up is cp
+    # (eta = 1); once it is exposed the speed-up is below cp and falls as the
+    # link gets slower (the page's validation criteria).
+    B, S, dqk, dv, R, c_kv = 1, 1 << 17, 192, 128, 1e15, 576
+    t1 = prefill_time_s(prefill_compute_time_s(B, S, dqk, dv, 1, R),
+                        pass_kv_bytes_per_chip(1, S, c_kv) / 1e9)
+    for cp in (2, 4, 8, 16):
+        t_comp = prefill_compute_time_s(B, S, dqk, dv, cp, R)
+        prev = None
+        for bw in (1e12, 1e9, 1e6, 1e5, 1e4, 1e3):
+            t_kv = pass_kv_bytes_per_chip(cp, S, c_kv) / bw
+            t = prefill_time_s(t_comp, t_kv)
+            eta = scaling_efficiency(t1, t, cp)
+            speedup = t1 / t
+            if t_kv <= t_comp:
+                assert eta == pytest.approx(1.0) and speedup == pytest.approx(cp)
+            else:
+                assert speedup < cp and eta < 1
+                assert prev is None or speedup < prev
+                prev = speedup
+        assert prev is not None             # the sweep reached the exposed regime
+    assert scaling_efficiency(3.0, 3.0, 1) == 1.0
