@@ -373,6 +373,6 @@ def pass_q_decode(q, k_shard, v_shard, scale=None, src=0, group=None, transport=
         o_p.zero_()
         l_p.fill_(float("-inf"))
     transport.all_gather(gathered, slot)
-    o_parts = gathered[:, :n_o].reshape(P, B, Hq, dv)
-    l_parts = gathered[:, n_o:].reshape(P, B, Hq)
+    o_parts = gathered[:, :n_o].contiguous().view(P, B, Hq, dv)
+    l_parts = gathered[:, n_o:].contiguous().view(P, B, Hq)
     return blocks.decode_merge(o_parts, l_parts, q.dtype)

@@ -31,7 +31,8 @@ def _free_port():
 
 
 class OracleBlocks:
-    """Block arithmetic from the oracle, for CPU tensors."""
+    """Block arithmetic from the oracle, for CPU tensors.  Like the library's
+    bindings, the merges take densely stacked partials only."""
 
     @staticmethod
     def _pos(off, stride, n):
@@ -47,6 +48,7 @@ class OracleBlocks:
 
     def merge(self, o_parts, lse_parts, out_dtype):
         from oracle.merge import lse_merge
+        assert o_parts.is_contiguous() and lse_parts.is_contiguous()
         oo, ll = lse_merge(o_parts.double().numpy(), lse_parts.double().numpy())
         return torch.from_numpy(oo).to(out_dtype), torch.from_numpy(ll).float()
 
