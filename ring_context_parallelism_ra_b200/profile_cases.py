@@ -12,6 +12,8 @@ kernel at a shape the bench uses, holding at most a few GB on the device:
                  1M-token cache (B = 4, 64/8 heads): one chunk-kernel launch
                  and one merge launch, as one shard of the bench's decode step
   merge_p8       LSE merge of 8 fp32 partials of shape [1, 32, 16384, 128]
+  merge_p4_8k    LSE merge of 4 fp32 partials of shape [1, 8, 2048, 128] (the
+                 partials one query partition of the 8K MHA ring collects)
   backward_cfg2  ring backward (prep, tensor-core kernel, dQ conversion) on the
                  bench's default workload, from its own forward O and LSE
   backward_gqa32k ring backward, causal GQA 32/8 heads, n = 32768, P = 8
@@ -47,7 +49,7 @@ def _backward(q, k, v, P, reps):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["prefill_cfg2", "prefill_gqa32k", "decode_shard", "merge_p8",
-                                     "backward_cfg2", "backward_gqa32k"])
+                                     "merge_p4_8k", "backward_cfg2", "backward_gqa32k"])
     ap.add_argument("--reps", type=int, default=1)
     args = ap.parse_args()
     dev = "cuda"
@@ -74,11 +76,12 @@ def main():
             ra.decode_partial(q, k, v, 0, 131072, None, ws, o, l)
         torch.cuda.synchronize()
     else:
+        P, H, L = (8, 32, 16384) if args.case == "merge_p8" else (4, 8, 2048)
         g = torch.Generator(device=dev).manual_seed(5)
-        o = torch.randn((8, 1, 32, 16384, 128), device=dev, generator=g)
-        l = torch.randn((8, 1, 32, 16384), device=dev, generator=g)
-        out = torch.empty((1, 32, 16384, 128), device=dev, dtype=torch.bfloat16)
-        lse = torch.empty((1, 32, 16384), device=dev)
+        o = torch.randn((P, 1, H, L, 128), device=dev, generator=g)
+        l = torch.randn((P, 1, H, L), device=dev, generator=g)
+        out = torch.empty((1, H, L, 128), device=dev, dtype=torch.bfloat16)
+        lse = torch.empty((1, H, L), device=dev)
         for _ in range(2 + args.reps):
             ra.lse_merge(o, l, torch.bfloat16, out, lse)
         torch.cuda.synchronize()
