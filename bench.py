@@ -9,7 +9,8 @@ API from pinned host buffers, the oracle's CPU throughput on a bounded
 sample, and the pass-Q decode leg (GB/s of KV cache read) that the metric
 also names.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2|3|5|1]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload causal_mha_8k|causal_gqa_128k|causal_mla_256k|noncausal_fp32_512]
     python bench.py --impl reference ...   # the fp64 CPU oracle, same line
 
 N > 1 (torchrun): every rank runs an independent replica of the workload
@@ -289,12 +290,12 @@ def run_ours(args, world, rank):
     torch.cuda.empty_cache()
 
     decode = None if args.skip_decode else run_decode_leg(args, world, rank, peaks, peaks_kind)
-    striped = None if args.skip_striped else run_striped_leg(args, world, rank, workload(3), peaks)
+    striped = None if args.skip_striped else run_striped_leg(args, world, rank, workload("causal_gqa_128k"), peaks)
     merge = None if args.skip_merge else run_merge_leg(args, world, rank, peaks, peaks_kind)
     backward = None
     if not args.skip_backward and wl.dtype == "bf16":
         backward = [run_backward_leg(args, world, rank, w, peaks, peaks_kind)
-                    for w in (wl, workload(3))]
+                    for w in (wl, workload("causal_gqa_128k"))]
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -332,7 +333,7 @@ def run_merge_leg(args, world, rank, peaks, peaks_kind):
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     stream = torch.cuda.current_stream()
     res = []
-    for key in (2, 3):
+    for key in ("causal_mha_8k", "causal_gqa_128k"):
         wl = workload(key)
         L = wl.n // wl.P
         g = torch.Generator(device=dev).manual_seed(wl.seed + 7 + 1000 * rank)
@@ -518,7 +519,7 @@ def run_striped_leg(args, world, rank, wl, peaks):
 
 def run_decode_leg(args, world, rank, peaks, peaks_kind):
     """Pass-Q decode over the 1M-token cache (P shards + merge): GB/s of K/V read."""
-    wl = workload(4)
+    wl = workload("decode_1m")
     dev = torch.device("cuda")
     q, k, v = make_workload_inputs(wl, device=dev)
     P = wl.P
@@ -595,7 +596,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 5])
+    ap.add_argument("--workload", default="causal_mha_8k",
+                    choices=["causal_mha_8k", "causal_gqa_128k", "causal_mla_256k",
+                             "noncausal_fp32_512"])
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-striped", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")

@@ -70,8 +70,8 @@ typedef struct {
  */
 
 /*
- * ra_block_partial -- one (Q range, KV range) block: the partial of step a3 of
- * the method, page "LLM长文本推理Ring Attention环形注意力机制实现与优化", section
+ * ra_block_partial -- one (Q range, KV range) block: the block partial of one
+ * ring step, page "LLM长文本推理Ring Attention环形注意力机制实现与优化", section
  * "Ring Attention实现代码与通信重叠" (each ring step computes the local
  * attention of Q_i against the KV block that has arrived).
  *   q, k, v     : device, BHSD as above (k, v hold the n_k keys of the block).
@@ -106,8 +106,8 @@ int ra_block_partial_strided(const void* q, const void* k, const void* v, const 
                              float* o_part, float* lse_part, void* stream);
 
 /*
- * ra_lse_merge -- N-way merge of normalised partials over disjoint key sets
- * (step a6), the closed form of the beta / gamma update of page
+ * ra_lse_merge -- N-way merge of normalised partials over disjoint key sets,
+ * the closed form of the beta / gamma update of page
  * "LLM长文本推理Ring Attention环形注意力机制实现与优化", section
  * "Ring Attention实现代码与通信重叠":
  *   L* = max_p L_p,  w_p = exp(L_p - L*),  LSE = L* + ln sum w_p,
@@ -124,7 +124,8 @@ int ra_lse_merge(const float* o_parts, const float* lse_parts, int P, const ra_s
 
 /*
  * ra_ring_forward -- the fused ring: all P partitions of one sequence in one
- * kernel (steps a1-a5).  Query partition i meets KV partitions in ring order
+ * kernel (split, ring schedule, block partials, fold and final normalisation).
+ * Query partition i meets KV partitions in ring order
  * j = i, i-1, ..., i-P+1 (mod P); with causal = 1 the blocks j > i are
  * skipped and the diagonal block is masked.  K/V tiles stream through a
  * shared-memory ring filled by TMA while the previous tile's math runs.
@@ -158,7 +159,7 @@ int ra_ring_forward_striped(const void* q, const void* k, const void* v, int P, 
 size_t ra_decode_workspace_bytes(const ra_shape* shape);
 
 /*
- * ra_decode_partial -- pass-Q decode on one KV shard (step a7), page
+ * ra_decode_partial -- pass-Q decode on one KV shard, page
  * "上下文并行 (CP) 收益评估实验设计", decode section: the query is sent to every
  * shard, each shard computes partial attention over its S/cp tokens, and the
  * partials are reduced (ra_decode_merge).  One query token per sequence sees
@@ -207,7 +208,7 @@ int ra_decode_partial_noalloc(const void* q, const void* k_shard, const void* v_
                               float* o_part, float* lse_part, void* stream);
 
 /*
- * ra_decode_merge -- reduce the P shard partials of pass-Q decode (step a8);
+ * ra_decode_merge -- reduce the P shard partials of pass-Q decode;
  * the merge of ra_lse_merge with n_q = 1.
  *   o_parts     : device fp32 [P, B, Hq, d_v];  lse_parts: [P, B, Hq].
  *   out         : device [B, Hq, d_v] of out_dtype;  lse: fp32 [B, Hq] or NULL.

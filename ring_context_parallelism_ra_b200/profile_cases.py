@@ -5,7 +5,7 @@
 Each case runs two warm-up launches and then N (default 1) launches of one
 kernel at a shape the bench uses, holding at most a few GB on the device:
 
-  prefill_cfg2   fused ring forward, causal MHA, 8 heads, n = 8192, d = 128,
+  prefill_mha8k   fused ring forward, causal MHA, 8 heads, n = 8192, d = 128,
                  P = 4 (the bench's default workload, one launch per step)
   prefill_gqa32k fused ring forward, causal GQA 32/8 heads, n = 32768, P = 8
   decode_shard   pass-Q decode partial on one 131072-token shard of the
@@ -14,7 +14,7 @@ kernel at a shape the bench uses, holding at most a few GB on the device:
   merge_p8       LSE merge of 8 fp32 partials of shape [1, 32, 16384, 128]
   merge_p4_8k    LSE merge of 4 fp32 partials of shape [1, 8, 2048, 128] (the
                  partials one query partition of the 8K MHA ring collects)
-  backward_cfg2  ring backward (prep, tensor-core kernel, dQ conversion) on the
+  backward_mha8k  ring backward (prep, tensor-core kernel, dQ conversion) on the
                  bench's default workload, from its own forward O and LSE
   backward_gqa32k ring backward, causal GQA 32/8 heads, n = 32768, P = 8
 """
@@ -48,20 +48,20 @@ def _backward(q, k, v, P, reps):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["prefill_cfg2", "prefill_gqa32k", "decode_shard", "merge_p8",
-                                     "merge_p4_8k", "backward_cfg2", "backward_gqa32k"])
+    ap.add_argument("case", choices=["prefill_mha8k", "prefill_gqa32k", "decode_shard", "merge_p8",
+                                     "merge_p4_8k", "backward_mha8k", "backward_gqa32k"])
     ap.add_argument("--reps", type=int, default=1)
     args = ap.parse_args()
     dev = "cuda"
-    if args.case == "prefill_cfg2":
-        wl = workload(2)
+    if args.case == "prefill_mha8k":
+        wl = workload("causal_mha_8k")
         q, k, v = make_workload_inputs(wl, device=dev)
         _prefill(q, k, v, wl.P, args.reps)
     elif args.case == "prefill_gqa32k":
         q, k, v = make_qkv(1, 32, 8, 32768, 32768, 128, 128, torch.bfloat16, seed=3, device=dev)
         _prefill(q, k, v, 8, args.reps)
-    elif args.case == "backward_cfg2":
-        wl = workload(2)
+    elif args.case == "backward_mha8k":
+        wl = workload("causal_mha_8k")
         q, k, v = make_workload_inputs(wl, device=dev)
         _backward(q, k, v, wl.P, args.reps)
     elif args.case == "backward_gqa32k":

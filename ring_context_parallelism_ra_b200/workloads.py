@@ -34,7 +34,7 @@ _TENSOR_ID = {"q": 1, "k": 2, "v": 3, "do": 4}
 
 @dataclass(frozen=True)
 class Workload:
-    key: int
+    key: str
     name: str
     B: int
     Hq: int
@@ -62,20 +62,22 @@ class Workload:
         return 1 if self.decode else self.n
 
 
-WORKLOADS = {
-    1: Workload(1, "noncausal_fp32_b1_h1_n512_d64_P4", 1, 1, 1, 512, 64, 64, "f32", 4, False, seed=1001),
-    2: Workload(2, "causal_mha_b1_h8_n8192_d128_P4", 1, 8, 8, 8192, 128, 128, "bf16", 4, True,
-                qk_mult=0.5, seed=1002),
-    3: Workload(3, "causal_gqa_b1_h32kv8_n131072_d128_P8", 1, 32, 8, 131072, 128, 128, "bf16", 8, True,
-                seed=1003),
-    4: Workload(4, "decode_passq_b4_h64kv8_n1048576_d128_P8", 4, 64, 8, 1048576, 128, 128, "bf16", 8,
-                False, decode=True, seed=1004),
-    5: Workload(5, "causal_mla_b1_h16_n262144_dqk192_dv128_P16", 1, 16, 16, 262144, 192, 128, "bf16",
-                16, True, seed=1005),
-}
+WORKLOADS = {w.key: w for w in (
+    Workload("noncausal_fp32_512", "noncausal_fp32_b1_h1_n512_d64_P4",
+             1, 1, 1, 512, 64, 64, "f32", 4, False, seed=1001),
+    Workload("causal_mha_8k", "causal_mha_b1_h8_n8192_d128_P4",
+             1, 8, 8, 8192, 128, 128, "bf16", 4, True, qk_mult=0.5, seed=1002),
+    Workload("causal_gqa_128k", "causal_gqa_b1_h32kv8_n131072_d128_P8",
+             1, 32, 8, 131072, 128, 128, "bf16", 8, True, seed=1003),
+    Workload("decode_1m", "decode_passq_b4_h64kv8_n1048576_d128_P8",
+             4, 64, 8, 1048576, 128, 128, "bf16", 8, False, decode=True, seed=1004),
+    Workload("causal_mla_256k", "causal_mla_b1_h16_n262144_dqk192_dv128_P16",
+             1, 16, 16, 262144, 192, 128, "bf16", 16, True, seed=1005),
+)}
 
 
-def workload(key: int) -> Workload:
+def workload(key: str) -> Workload:
+    """The workload registered under `key` (one of ``WORKLOADS``)."""
     return WORKLOADS[key]
 
 

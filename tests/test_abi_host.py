@@ -91,6 +91,14 @@ def test_validation_rejects_bad_arguments_before_launch():
     sd3 = _shape(n_q=1, Hq=8, Hkv=1, n_k=4096, d_qk=64, d_v=64)
     assert L.ra_decode_partial(p, p, p, 4096, ctypes.byref(sd3), 1.0, p, p, p, 1 << 30, nul) == UNS
     assert L.ra_decode_merge(p, p, 2, ctypes.byref(_shape(n_q=4)), p, 0, p, nul) == INV
+    # empty inputs are rejected, not launched: no sequence, no batch, no heads
+    s0 = _shape(n_q=0, n_k=0)
+    assert L.ra_ring_forward(p, p, p, 1, 1, 1.0, p, p, ctypes.byref(s0), nul) == INV
+    assert L.ra_block_partial(p, p, p, ctypes.byref(_shape(n_k=0)), 0, 0, 1, 1.0, p, p, nul) == INV
+    assert L.ra_block_partial(p, p, p, ctypes.byref(_shape(B=0)), 0, 0, 1, 1.0, p, p, nul) == INV
+    assert L.ra_lse_merge(p, p, 2, ctypes.byref(_shape(Hq=0, Hkv=0)), p, 0, p, nul) == INV
+    assert L.ra_decode_partial(p, p, p, 0, ctypes.byref(_shape(n_q=1, Hq=8, Hkv=1, n_k=0)), 1.0,
+                               p, p, p, 1 << 30, nul) == INV
     out = np.empty(4, dtype=np.int8)
     assert L.ra_block_class(0, 4, 1, 1, 0, 0, 1, out.ctypes.data_as(ctypes.c_void_p)) == INV
     assert L.ra_block_class(4, 4, 0, 1, 0, 0, 1, out.ctypes.data_as(ctypes.c_void_p)) == INV

@@ -53,7 +53,7 @@ def test_max_over_ranks_gloo_world2():
 
 
 def test_replica_seeds_give_different_inputs():
-    wl = workload(1)
+    wl = workload("noncausal_fp32_512")
     q0, _, _ = make_workload_inputs(wl)
     q1, _, _ = make_workload_inputs(dataclasses.replace(wl, seed=wl.seed + 1000))
     q0b, _, _ = make_workload_inputs(wl)
@@ -83,7 +83,7 @@ def test_reference_arm_line():
         assert key in line
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
-    assert line["config"]["workload"] == workload(2).name
+    assert line["config"]["workload"] == workload("causal_mha_8k").name
 
 
 def test_flop_and_byte_counts_match_oracle_formulas():
@@ -91,12 +91,12 @@ def test_flop_and_byte_counts_match_oracle_formulas():
     from oracle.costs import kv_cache_bytes, prefill_flops as oracle_flops
     from ring_context_parallelism_ra_b200.workloads import (backward_flops, decode_kv_bytes,
                                                            prefill_flops)
-    for key in (1, 2, 3, 5):
+    for key in ("noncausal_fp32_512", "causal_mha_8k", "causal_gqa_128k", "causal_mla_256k"):
         wl = workload(key)
         assert prefill_flops(wl) == oracle_flops(wl.B, wl.n, wl.d_qk, wl.d_v, wl.Hq, wl.causal)
         assert backward_flops(wl) == oracle_bwd_flops(wl.B, wl.n, wl.d_qk, wl.d_v, wl.Hq,
                                                       wl.causal)
-    wl = workload(4)
+    wl = workload("decode_1m")
     assert decode_kv_bytes(wl) == wl.B * kv_cache_bytes(1, wl.Hkv, wl.d_qk, wl.n, 2)
     assert decode_kv_bytes(wl) == 17179869184
 

@@ -189,7 +189,7 @@ def test_backward_sampled_at_8k_mha_workload():
     # The 8K causal MHA workload (8 heads, d 128, P 4, Q and K scaled by 0.5),
     # the configuration the bench times: exact gradients on sampled rows / keys
     # of every head, plus identities over all keys.
-    wl = workload(2)
+    wl = workload("causal_mha_8k")
     q, k, v = make_qkv(wl.B, wl.Hq, wl.Hkv, wl.n, wl.n, wl.d_qk, wl.d_v, BF, seed=wl.seed,
                        qk_mult=wl.qk_mult, device=DEV)
     g = make_dout(wl.B, wl.Hq, wl.n, wl.d_v, BF, seed=wl.seed, device=DEV)

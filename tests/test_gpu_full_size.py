@@ -34,7 +34,7 @@ def sample_rows(n, P, tile=128, n_uniform=64, seed=0):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-def _check_prefill(key, heads):
+def _check_prefill(key, heads, row_seed):
     wl = workload(key)
     torch.cuda.empty_cache()
     q, k, v = make_workload_inputs(wl, device="cuda")
@@ -42,7 +42,7 @@ def _check_prefill(key, heads):
     assert ra.get_status() == ra.RA_OK
     assert torch.isfinite(out).all().item()
     assert torch.isfinite(lse).all().item()
-    rows = sample_rows(wl.n, wl.P, seed=key)
+    rows = sample_rows(wl.n, wl.P, seed=row_seed)
     G = wl.Hq // wl.Hkv
     q_s = q[:, heads].cpu()
     k_s = torch.stack([k[:, h // G] for h in heads], dim=1).cpu()
@@ -57,16 +57,16 @@ def _check_prefill(key, heads):
     torch.cuda.empty_cache()
 
 
-def test_config3_causal_gqa_128k():
-    _check_prefill(3, heads=[0, 3, 4, 31])
+def test_causal_gqa_128k_full_size():
+    _check_prefill("causal_gqa_128k", heads=[0, 3, 4, 31], row_seed=3)
 
 
-def test_config5_causal_mla_256k():
-    _check_prefill(5, heads=[0, 15])
+def test_causal_mla_256k_full_size():
+    _check_prefill("causal_mla_256k", heads=[0, 15], row_seed=5)
 
 
-def test_config4_decode_pass_q_1m():
-    wl = workload(4)
+def test_decode_pass_q_1m_full_size():
+    wl = workload("decode_1m")
     torch.cuda.empty_cache()
     q, k, v = make_workload_inputs(wl, device="cuda")
     out, lse = ra.decode_pass_q(q, k, v, wl.P, wl.scale)
@@ -85,7 +85,7 @@ def test_config4_decode_pass_q_1m():
     torch.cuda.empty_cache()
 
 
-def test_config3_backward_gqa_128k():
+def test_backward_causal_gqa_128k_full_size():
     # The ring backward on the causal GQA 128K workload in the bench's
     # configuration: exact gradients on sampled query rows (dQ) and on the
     # last 256 keys (dK, dV; a causal key u needs only rows t >= u), for the
@@ -94,7 +94,7 @@ def test_config3_backward_gqa_128k():
     from oracle.backward import attention_backward_sampled
     from ring_context_parallelism_ra_b200.workloads import make_dout
     from tests.parity_util import check_grad, to64
-    wl = workload(3)
+    wl = workload("causal_gqa_128k")
     torch.cuda.empty_cache()
     q, k, v = make_workload_inputs(wl, device="cuda")
     g = make_dout(wl.B, wl.Hq, wl.n, wl.d_v, wl.torch_dtype, seed=wl.seed, device="cuda")

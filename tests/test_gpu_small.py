@@ -195,8 +195,8 @@ def test_causal_output_ignores_future_tokens(dt):
     assert torch.equal(l1[:, :, :t + 1], l2[:, :, :t + 1])
 
 
-def test_config1_full_fp32():
-    wl = workload(1)
+def test_noncausal_fp32_512_full():
+    wl = workload("noncausal_fp32_512")
     q, k, v = make_workload_inputs(wl)
     out, lse = ra.ring_forward(q.to(DEV), k.to(DEV), v.to(DEV), wl.P, wl.causal, wl.scale)
     want_o, want_l = oracle_attention(q, k, v, wl.scale, wl.causal)
@@ -204,8 +204,8 @@ def test_config1_full_fp32():
     check_lse(lse, want_l)
 
 
-def test_config2_full_bf16():
-    wl = workload(2)
+def test_causal_mha_8k_full_bf16():
+    wl = workload("causal_mha_8k")
     q, k, v = make_workload_inputs(wl)
     out, lse = ra.ring_forward(q.to(DEV), k.to(DEV), v.to(DEV), wl.P, wl.causal, wl.scale)
     want_o, want_l = oracle_attention(q, k, v, wl.scale, wl.causal)
