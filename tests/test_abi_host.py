@@ -4,9 +4,12 @@ behaves, without launching anything on a GPU."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import numpy as np
 import pytest
+import torch
 
 from oracle.block_class import block_class as oracle_block_class
 from oracle.block_class import partition_class
@@ -163,3 +166,30 @@ def test_backward_workspace_size():
         rows = B * H * ((n + 127) // 128) * 128
         got = ra.lib().ra_backward_workspace_bytes(ctypes.byref(s))
         assert rows * (d + 2) * 4 <= got < rows * (d + 2) * 4 + 1024
+
+
+def test_no_cpu_fallback_cpu_tensors_are_rejected():
+    # the binding only marshals device pointers: CPU tensors are an error,
+    # never a silent host computation
+    q = torch.zeros((1, 1, 128, 64), dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        ra.ring_forward(q, q, q, 1, True)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        ra.lse_merge(torch.zeros((2, 1, 1, 4, 64)), torch.zeros((2, 1, 1, 4)), torch.float32)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # with the compiled library absent the package raises on first use
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from ring_context_parallelism_ra_b200 import ra\n"
+        "ra.library_path = lambda: %r\n"
+        "try:\n"
+        "    ra.lib()\n"
+        "except RuntimeError as e:\n"
+        "    print('raised:', e)\n"
+        "    sys.exit(0)\n"
+        "sys.exit(3)\n" % (ROOT, str(tmp_path / "libra.so")))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "is missing" in r.stdout
