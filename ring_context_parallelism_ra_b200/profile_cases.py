@@ -3,7 +3,9 @@
     python -m ring_context_parallelism_ra_b200.profile_cases CASE [--reps N]
 
 Each case runs two warm-up launches and then N (default 1) launches of one
-kernel at a shape the bench uses, holding at most a few GB on the device:
+kernel at a shape the bench uses, holding at most a few GB on the device
+(``--activity``: the same launches recorded by torch.profiler, each
+kernel's device time printed; no replay, unlike ncu):
 
   prefill_mha8k   fused ring forward, causal MHA, 8 heads, n = 8192, d = 128,
                  P = 4 (the bench's default workload, one launch per step)
@@ -28,10 +30,23 @@ from . import ra
 from .workloads import make_dout, make_qkv, make_workload_inputs, workload
 
 
+# With --activity every launch starts from a cold L2, as in the bench: a
+# 256 MiB buffer is written before it.
+_FLUSH = {"on": False, "buf": None}
+
+
+def _flush():
+    if _FLUSH["on"]:
+        if _FLUSH["buf"] is None:
+            _FLUSH["buf"] = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        _FLUSH["buf"].zero_()
+
+
 def _prefill(q, k, v, P, reps):
     out = torch.empty((*q.shape[:3], v.shape[-1]), device=q.device, dtype=q.dtype)
     lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
     for _ in range(2 + reps):
+        _flush()
         ra.ring_forward(q, k, v, P, True, None, out, lse)
     torch.cuda.synchronize()
 
@@ -42,6 +57,7 @@ def _backward(q, k, v, P, reps):
     ws = torch.empty(ra.backward_workspace_bytes(q, k, v), dtype=torch.uint8, device=q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     for _ in range(2 + reps):
+        _flush()
         ra.ring_backward(q, k, v, out, lse, g, P, True, None, dq, dk, dv, ws)
     torch.cuda.synchronize()
 
@@ -51,7 +67,24 @@ def main():
     ap.add_argument("case", choices=["prefill_mha8k", "prefill_gqa32k", "decode_shard", "merge_p8",
                                      "merge_p4_8k", "backward_mha8k", "backward_gqa32k"])
     ap.add_argument("--reps", type=int, default=1)
+    ap.add_argument("--activity", action="store_true",
+                    help="record the launches with torch.profiler (kernel activity records, "
+                         "no replay) and print each kernel's device time")
     args = ap.parse_args()
+    if args.activity:
+        from torch.profiler import ProfilerActivity, profile
+        _FLUSH["on"] = True
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            run_case(args)
+        print(prof.key_averages().table(sort_by="cuda_time_total", row_limit=12,
+                                        max_name_column_width=70))
+    else:
+        run_case(args)
+    assert ra.get_status() == ra.RA_OK
+    print(f"{args.case}: ok")
+
+
+def run_case(args):
     dev = "cuda"
     if args.case == "prefill_mha8k":
         wl = workload("causal_mha_8k")
@@ -83,10 +116,9 @@ def main():
         out = torch.empty((1, H, L, 128), device=dev, dtype=torch.bfloat16)
         lse = torch.empty((1, H, L), device=dev)
         for _ in range(2 + args.reps):
+            _flush()
             ra.lse_merge(o, l, torch.bfloat16, out, lse)
         torch.cuda.synchronize()
-    assert ra.get_status() == ra.RA_OK
-    print(f"{args.case}: ok")
 
 
 if __name__ == "__main__":
