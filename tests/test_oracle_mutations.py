@@ -1,0 +1,227 @@
+"""Planted mistakes in the oracle (CPU only).
+
+Each case loads a copy of one oracle module with one plausible mistake
+written into its source (a dropped term, a wrong sign, an off-by-one mask, a
+wrong head map, a swapped operand), runs that module's pins against the
+copy, and requires at least one pin to fail.  The same pins hold for the
+unmodified oracle (the ``test_oracle_*`` files); this file shows that they
+would notice such a mistake.
+
+A mutation that cannot change any result (an equivalent rewrite) is not
+listed: clearing rows whose weights are already zero, or transposing a
+product twice, leaves every output as it was.
+"""
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+import torch
+
+from tests.test_oracle_attention import CASES, _brute
+from tests.test_oracle_backward import FD_CASES, _fd_grad, _inputs, _torch_attention
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _mutant(module, old, new):
+    """oracle/<module>.py with `old` replaced by `new` (every occurrence),
+    loaded as a module of the oracle package (its relative imports resolve to
+    the unmodified modules)."""
+    path = os.path.join(ROOT, "oracle", module + ".py")
+    src = open(path).read()
+    assert old in src, f"mutation site not found in oracle/{module}.py: {old!r}"
+    mod = types.ModuleType(f"oracle._mutant_{module}")
+    mod.__package__ = "oracle"
+    exec(compile(src.replace(old, new), path, "exec"), mod.__dict__)  # noqa: S102
+    return mod
+
+
+def _holds(check, *args):
+    """True when the pin holds for the function under test; an exception
+    (a shape error from a wrong operand, say) counts as a failed pin."""
+    try:
+        check(*args)
+        return True
+    except Exception:  # noqa: BLE001
+        return False
+
+
+# ------------------------------------------------------------ attention --
+
+def _pin_brute_force(att):
+    for case in CASES:
+        B, hq, hkv, nq, nk, d, dv, causal, qo, ko = case
+        rng = np.random.default_rng(abs(hash(case)) % 2**32)
+        q = rng.standard_normal((B, hq, nq, d))
+        k = rng.standard_normal((B, hkv, nk, d))
+        v = rng.standard_normal((B, hkv, nk, dv))
+        o, lse = att(q, k, v, 0.6, causal, q_offset=qo, k_offset=ko)
+        wo, wl = _brute(q, k, v, 0.6, causal, qo, ko)
+        assert np.allclose(o, wo, atol=1e-12, rtol=0)
+        fin = np.isfinite(wl)
+        assert (np.isfinite(lse) == fin).all()
+        assert np.allclose(lse[fin], wl[fin], atol=1e-12, rtol=0)
+
+
+def _pin_zero_query(att):
+    rng = np.random.default_rng(3)
+    n = 9
+    q = np.zeros((1, 1, n, 4))
+    k = rng.standard_normal((1, 1, n, 4))
+    v = rng.standard_normal((1, 1, n, 3))
+    o, lse = att(q, k, v, 0.8, True)
+    for t in range(n):
+        assert abs(lse[0, 0, t] - math.log(t + 1)) <= 1e-12
+        assert np.abs(o[0, 0, t] - v[0, 0, :t + 1].mean(axis=0)).max() <= 1e-12
+
+
+def _pin_causal_independence(att):
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.standard_normal((1, 2, 10, 3)) for _ in range(3))
+    o1, _ = att(q, k, v, 0.5, True)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, 6:] += 5.0
+    v2[:, :, 6:] -= 3.0
+    o2, _ = att(q, k2, v2, 0.5, True)
+    assert np.array_equal(o1[:, :, :6], o2[:, :, :6])
+
+
+ATTENTION_PINS = [_pin_brute_force, _pin_zero_query, _pin_causal_independence]
+
+ATTENTION_MUTANTS = {
+    "scale dropped": ("(q_rows @ k.T) * scale", "(q_rows @ k.T)"),
+    "mask off by one": ("k_pos[None, :] <= q_pos[:, None]", "k_pos[None, :] < q_pos[:, None]"),
+    "mask reversed": ("k_pos[None, :] <= q_pos[:, None]", "q_pos[:, None] <= k_pos[None, :]"),
+    "interleaved GQA map": ("g = h // grp", "g = h % h_kv"),
+    "LSE in base 2": ("m_safe + np.log(", "m_safe + np.log2("),
+    "max added, not subtracted": ("np.exp(s - m_safe[:, None])", "np.exp(s + m_safe[:, None])"),
+    "normalisation dropped": ("o = (e @ v) / np.where(empty, 1.0, z)[:, None]", "o = (e @ v)"),
+    "query offset taken from keys": ("q_offset + np.arange(n_q", "k_offset + np.arange(n_q"),
+}
+
+
+def test_attention_pins_hold_for_the_oracle():
+    from oracle.attention import attention
+    assert all(_holds(p, attention) for p in ATTENTION_PINS)
+
+
+@pytest.mark.parametrize("name", sorted(ATTENTION_MUTANTS))
+def test_attention_pins_catch_planted_mistake(name):
+    old, new = ATTENTION_MUTANTS[name]
+    att = _mutant("attention", old, new).attention
+    assert not all(_holds(p, att) for p in ATTENTION_PINS), name
+
+
+# ---------------------------------------------------------------- merge --
+
+def _pin_merge_equals_full(merge):
+    from oracle.attention import attention
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((1, 2, 7, 4))
+    k = rng.standard_normal((1, 2, 12, 4))
+    v = rng.standard_normal((1, 2, 12, 3))
+    want_o, want_l = attention(q, k, v, 0.7, False)
+    parts = [attention(q, k[:, :, a:b], v[:, :, a:b], 0.7, False) for a, b in ((0, 3), (3, 8), (8, 12))]
+    o, lse = merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    assert np.abs(o - want_o).max() <= 1e-12 and np.abs(lse - want_l).max() <= 1e-12
+
+
+def _pin_merge_empty(merge):
+    o, lse = merge(np.ones((2, 3, 4)), np.full((2, 3), -np.inf))
+    assert (o == 0).all() and (lse == -np.inf).all()
+    o1 = np.arange(4.0)
+    for parts, lses in (([o1, 7 * np.ones(4)], [0.3, -np.inf]),
+                        ([7 * np.ones(4), o1], [-np.inf, 0.3])):   # empty partial first
+        o, lse = merge(np.stack(parts), np.array(lses))
+        assert np.array_equal(o, o1) and lse == 0.3
+
+
+def _pin_merge_equal_halves(merge):
+    a, b = np.array([1.0, -2.0]), np.array([3.0, 4.0])
+    o, lse = merge(np.stack([a, b]), np.array([1.5, 1.5]))
+    assert np.abs(o - (a + b) / 2).max() <= 1e-15 and abs(lse - (1.5 + math.log(2))) <= 1e-15
+
+
+MERGE_PINS = [_pin_merge_equals_full, _pin_merge_empty, _pin_merge_equal_halves]
+
+MERGE_MUTANTS = {
+    "weight exponent negated": ("w = np.exp(lse_parts - l_ref[None])", "w = np.exp(l_ref[None] - lse_parts)"),
+    "LSE without the sum": ("l_ref + np.log(safe)", "l_ref"),
+    "normalisation dropped": ("/ safe[..., None]", ""),
+    "first partial as the reference": ("l_star = lse_parts.max(axis=0)", "l_star = lse_parts[0]"),
+}
+
+
+def test_merge_pins_hold_for_the_oracle():
+    from oracle.merge import lse_merge
+    assert all(_holds(p, lse_merge) for p in MERGE_PINS)
+
+
+@pytest.mark.parametrize("name", sorted(MERGE_MUTANTS))
+def test_merge_pins_catch_planted_mistake(name):
+    old, new = MERGE_MUTANTS[name]
+    merge = _mutant("merge", old, new).lse_merge
+    assert not all(_holds(p, merge) for p in MERGE_PINS), name
+
+
+# ------------------------------------------------------------- backward --
+
+def _pin_finite_differences(bwd):
+    from oracle.attention import attention
+    for case in FD_CASES:
+        hq, hkv, nq, nk, causal, qo, ko = case
+        q, k, v, g = _inputs(abs(hash(case)) % 1000, hq=hq, hkv=hkv, nq=nq, nk=nk)
+        kw = dict(q_offset=qo, k_offset=ko)
+        dq, dk, dv = bwd(q, k, v, g, 0.7, causal, **kw)
+
+        def f():
+            return float((attention(q, k, v, 0.7, causal, **kw)[0] * g).sum())
+        for got, x in ((dq, q), (dk, k), (dv, v)):
+            want = _fd_grad(x, f)
+            assert np.abs(got - want).max() <= 1e-7 * max(1.0, np.abs(want).max())
+
+
+def _pin_autodiff(bwd):
+    q, k, v, g = _inputs(5, B=1, hq=4, hkv=2, nq=12, nk=12, d=5, dv=3)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    pos = torch.arange(12)
+    (_torch_attention(tq, tk, tv, 0.45, True, pos, pos) * torch.tensor(g)).sum().backward()
+    dq, dk, dv = bwd(q, k, v, g, 0.45, True, row_chunk=5)
+    for got, t in ((dq, tq), (dk, tk), (dv, tv)):
+        assert np.abs(got - t.grad.numpy()).max() <= 1e-12
+
+
+def _pin_identities(bwd):
+    q, k, v, g = _inputs(8, hq=4, hkv=2, nq=10, nk=10, d=5, dv=3)
+    _, dk, dv = bwd(q, k, v, g, 0.4, True)
+    assert np.abs(dk.sum(axis=2)).max() <= 1e-12
+    want = g.reshape(1, 2, 2, 10, 3).sum(axis=(2, 3))
+    assert np.abs(dv.sum(axis=2) - want).max() <= 1e-12
+
+
+BACKWARD_PINS = [_pin_finite_differences, _pin_autodiff, _pin_identities]
+
+BACKWARD_MUTANTS = {
+    "row term D dropped": ("ds = p * (dp - d_row[:, None])", "ds = p * dp"),
+    "scale dropped from dQ": ("dq[b, h, r] = scale * (ds @ kk)", "dq[b, h, r] = ds @ kk"),
+    "dK from P instead of dS": ("dk[b, g] += scale * (ds.T @ qh[r])", "dk[b, g] += scale * (p.T @ qh[r])"),
+    "dV overwritten across a group": ("dv[b, g] += p.T @ doh[r]", "dv[b, g] = p.T @ doh[r]"),
+    "D summed over the wrong axis": ("d_row = (doh[r] * o).sum(axis=1)", "d_row = (doh[r] * o).sum(axis=0)"),
+    "dS sign flipped": ("ds = p * (dp - d_row[:, None])", "ds = p * (d_row[:, None] - dp)"),
+}
+
+
+def test_backward_pins_hold_for_the_oracle():
+    from oracle.backward import attention_backward
+    assert all(_holds(p, attention_backward) for p in BACKWARD_PINS)
+
+
+@pytest.mark.parametrize("name", sorted(BACKWARD_MUTANTS))
+def test_backward_pins_catch_planted_mistake(name):
+    old, new = BACKWARD_MUTANTS[name]
+    bwd = _mutant("backward", old, new).attention_backward
+    assert not all(_holds(p, bwd) for p in BACKWARD_PINS), name
