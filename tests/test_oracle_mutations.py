@@ -225,3 +225,56 @@ def test_backward_pins_catch_planted_mistake(name):
     old, new = BACKWARD_MUTANTS[name]
     bwd = _mutant("backward", old, new).attention_backward
     assert not all(_holds(p, bwd) for p in BACKWARD_PINS), name
+
+
+# ------------------------------------------------------------ blockwise --
+
+def _pin_ring_equals_definition(mod):
+    from oracle.attention import attention
+    rng = np.random.default_rng(6)
+    q = rng.standard_normal((1, 4, 24, 5)) * 2.0     # wide score spread: maxima move
+    k = rng.standard_normal((1, 2, 24, 5)) * 2.0
+    v = rng.standard_normal((1, 2, 24, 3))
+    for causal in (True, False):
+        want_o, want_l = attention(q, k, v, 0.6, causal)
+        for P in (1, 2, 3, 4, 8):
+            for ring in (mod.ring_attention_normalised, mod.ring_attention_online):
+                o, lse = ring(q, k, v, P, 0.6, causal)
+                assert np.abs(o - want_o).max() <= 1e-12
+                assert np.abs(lse - want_l).max() <= 1e-12
+
+
+def _pin_ring_any_block_order(mod):
+    from oracle.attention import attention
+    rng = np.random.default_rng(7)
+    q, k, v = (rng.standard_normal((1, 1, 20, 4)) for _ in range(3))
+    want_o, _ = attention(q, k, v, 0.5, True)
+    perms = [list(rng.permutation(4)) for _ in range(4)]
+    for ring in (mod.ring_attention_normalised, mod.ring_attention_online):
+        o, _ = ring(q, k, v, 4, 0.5, True, order=lambda i: perms[i])
+        assert np.abs(o - want_o).max() <= 1e-12
+
+
+BLOCKWISE_PINS = [_pin_ring_equals_definition, _pin_ring_any_block_order]
+
+BLOCKWISE_MUTANTS = {
+    "beta exponent negated": ("np.exp(old_safe - new_lse)", "np.exp(new_lse - old_safe)"),
+    "gamma without the block sum": ("gamma = w_sum * np.exp(max_val - new_lse)",
+                                    "gamma = np.exp(max_val - new_lse)"),
+    "running sum not rescaled": ("l = alpha * l + p.sum(axis=1)", "l = l + p.sum(axis=1)"),
+    "accumulator not rescaled": ("acc = alpha[:, None] * acc + p @ v_blk", "acc = acc + p @ v_blk"),
+    "diagonal block skipped": ("if causal and k0 > q1 - 1:", "if causal and k0 >= q0:"),
+    "interleaved GQA map": ("g = h // grp", "g = h % h_kv"),
+}
+
+
+def test_blockwise_pins_hold_for_the_oracle():
+    import oracle.blockwise as mod
+    assert all(_holds(p, mod) for p in BLOCKWISE_PINS)
+
+
+@pytest.mark.parametrize("name", sorted(BLOCKWISE_MUTANTS))
+def test_blockwise_pins_catch_planted_mistake(name):
+    old, new = BLOCKWISE_MUTANTS[name]
+    mod = _mutant("blockwise", old, new)
+    assert not all(_holds(p, mod) for p in BLOCKWISE_PINS), name
