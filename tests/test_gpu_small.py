@@ -111,6 +111,12 @@ RING_CASES = [
     (1, 2, 2, 768, 192, 128, 3, True, torch.bfloat16),      # MLA-shaped head
     (1, 8, 2, 257, 128, 128, 1, True, torch.bfloat16),      # P = 1, ragged tail
     (1, 1, 1, 1, 128, 128, 1, True, torch.bfloat16),        # a single token
+    (1, 2, 1, 300, 64, 128, 3, True, torch.bfloat16),       # the other head-dim pairs
+    (1, 2, 2, 256, 128, 64, 2, True, torch.bfloat16),
+    (1, 2, 1, 384, 192, 64, 4, True, torch.bfloat16),
+    (1, 2, 2, 96, 128, 128, 8, True, torch.bfloat16),       # 12-token partitions
+    (1, 2, 1, 16, 128, 128, 16, True, torch.bfloat16),      # one token per partition
+    (1, 1, 1, 8, 64, 64, 8, True, torch.float32),
 ]
 
 
