@@ -50,6 +50,9 @@ RING_CASES = [
     (1, 1, 1, 512, 64, 64, 4, False, F32),    # shape of the fp32 correctness workload
     (1, 2, 1, 320, 128, 128, 2, True, F32),
     (1, 4, 2, 200, 64, 128, 4, True, F32),
+    (1, 2, 2, 96, 128, 128, 8, True, BF),     # 12-token partitions
+    (1, 2, 1, 16, 128, 128, 16, True, BF),    # one token per partition
+    (1, 1, 1, 1, 128, 128, 1, True, BF),      # a single token: every gradient is 0 but dV
 ]
 
 
