@@ -255,6 +255,13 @@ def run_ours(args, world, rank):
                 "traffic": tr["dram_bytes_per_launch"] if tr else None,
                 "peak_kind": f"{peaks_kind} bf16 burst", "kernel": "ring_forward",
                 "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", 1400.0), 4)}
+    if wl.dtype == "f32":  # the exact-fp32 path runs on the CUDA cores, not the tensor cores
+        mhz = clk.summary().get("sm_max_mhz") or 1965
+        num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        peak = alu_peak_tflops(mhz, num_sms)
+        roofline.update({"peak": round(peak, 2), "frac": round(achieved / peak, 4),
+                         "peak_kind": f"fp32 FMA: {num_sms} SMs x 128 lanes x 2 FLOP x {mhz} MHz",
+                         "frac_of_sustained": None})
 
     # end to end through the public API from pinned host buffers: every step
     # copies its inputs in and its output and LSE out, inside the timed
@@ -292,6 +299,8 @@ def run_ours(args, world, rank):
     decode = None if args.skip_decode else run_decode_leg(args, world, rank, peaks, peaks_kind)
     striped = None if args.skip_striped else run_striped_leg(args, world, rank, workload("causal_gqa_128k"), peaks)
     merge = None if args.skip_merge else run_merge_leg(args, world, rank, peaks, peaks_kind)
+    others = (None if args.skip_workloads
+              else run_workloads_leg(args, world, rank, args.workload, peaks, peaks_kind))
     backward = None
     if not args.skip_backward and wl.dtype == "bf16":
         backward = [run_backward_leg(args, world, rank, w, peaks, peaks_kind)
@@ -320,7 +329,79 @@ def run_ours(args, world, rank):
         line["backward"] = backward
     if merge is not None:
         line["merge"] = merge
+    if others is not None:
+        line["workloads"] = others
     return line
+
+
+def alu_peak_tflops(sm_mhz, num_sms):
+    """fp32 FMA peak of the CUDA cores (not the tensor cores): 128 fp32 lanes
+    per SM, 2 FLOP per FMA, at the given SM clock."""
+    return num_sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def run_workloads_leg(args, world, rank, main_key, peaks, peaks_kind):
+    """The fused ring forward on the other configured workloads (the fp32
+    correctness shape, causal GQA 128K, causal MLA 256K), each timed like the
+    main leg: warm-up, L2 flushed before every step, CUDA events on the
+    launching stream, SM clocks sampled while timing."""
+    dev = torch.device("cuda")
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    res = []
+    for key in ("noncausal_fp32_512", "causal_gqa_128k", "causal_mla_256k"):
+        if key == main_key:
+            continue
+        wl = workload(key)
+        flops = prefill_flops(wl)
+        q, k, v = make_workload_inputs(dataclasses.replace(wl, seed=wl.seed + 1000 * rank), device=dev)
+        out = torch.empty((wl.B, wl.Hq, wl.n, wl.d_v), device=dev, dtype=wl.torch_dtype)
+        lse = torch.empty((wl.B, wl.Hq, wl.n), device=dev)
+        steps = 10 if wl.n <= 8192 else 3
+        for _ in range(3):
+            flush.zero_()
+            ra.ring_forward(q, k, v, wl.P, wl.causal, wl.scale, out, lse)
+        torch.cuda.synchronize()
+        events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps)]
+        barrier(world)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            for e0, e1 in events:
+                flush.zero_()
+                e0.record(stream)
+                ra.ring_forward(q, k, v, wl.P, wl.causal, wl.scale, out, lse)
+                e1.record(stream)
+            torch.cuda.synchronize()
+        assert ra.get_status() == ra.RA_OK
+        ms_local = statistics.mean(e0.elapsed_time(e1) for e0, e1 in events)
+        ms = max_over_ranks(ms_local, world)
+        achieved = flops / (ms_local * 1e-3) / 1e12
+        clocks = clk.summary()
+        if wl.dtype == "bf16":
+            peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+            sus = peaks.get("bf16_tflops_sustained")
+            roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "frac_of_sustained": round(achieved / sus, 4) if sus else None,
+                    "peak_kind": f"{peaks_kind} bf16 burst", "kernel": "tc_attention_kernel"}
+        else:
+            mhz = clocks.get("sm_max_mhz") or 1965
+            peak = alu_peak_tflops(mhz, num_sms)
+            roof = {"bound": "alu", "achieved": round(achieved, 3), "peak": round(peak, 2),
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "peak_kind": f"fp32 FMA: {num_sms} SMs x 128 lanes x 2 FLOP x {mhz} MHz",
+                    "kernel": "simt_attention_kernel",
+                    "note": "correctness shape (512 tokens); its time is launch-dominated"}
+        res.append({"workload": wl.name, "value": round(world * flops / (ms * 1e-3) / 1e12, 3),
+                    "unit": "TFLOP/s", "ms_per_step": round(ms, 5), "steps": steps, "warmup": 3,
+                    "dtype": "bf16" if wl.dtype == "bf16" else "f32", "roofline": roof,
+                    "clocks": clocks})
+        del q, k, v, out, lse
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_merge_leg(args, world, rank, peaks, peaks_kind):
@@ -603,6 +684,7 @@ def main():
     ap.add_argument("--skip-striped", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--skip-merge", action="store_true")
+    ap.add_argument("--skip-workloads", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:
