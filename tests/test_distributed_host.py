@@ -271,3 +271,62 @@ def test_pass_q_decode_over_gloo_matches_whole_cache(sizes):
         errs.append(errq.get())
     assert not errs, errs
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+
+
+def _subgroup_main(rank, world, port, errq):
+    import torch.distributed as dist
+
+    from oracle.attention import attention
+    from ring_context_parallelism_ra_b200.distributed import (HostTransport, pass_q_decode,
+                                                              ring_attention_forward)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        # two independent rings, {0, 1} and {2, 3}, each on its own sequence:
+        # point-to-point calls need global ranks, the ring uses group ranks
+        groups = [dist.new_group([0, 1]), dist.new_group([2, 3])]
+        gi = rank // 2
+        grp, me = groups[gi], rank % 2
+        B, Hq, Hkv, L, d, dv = 1, 2, 1, 6, 4, 3
+        n = 2 * L
+        rng = np.random.default_rng(4000 + gi)
+        q = torch.from_numpy(rng.standard_normal((B, Hq, n, d)))
+        k = torch.from_numpy(rng.standard_normal((B, Hkv, n, d)))
+        v = torch.from_numpy(rng.standard_normal((B, Hkv, n, dv)))
+        rows = np.arange(me * L, (me + 1) * L)
+        part = lambda x: x[:, :, rows].contiguous()  # noqa: E731
+        out, lse = ring_attention_forward(part(q), part(k), part(v), True, 0.5, group=grp,
+                                          transport=HostTransport(grp), blocks=OracleBlocks())
+        want_o, want_l = attention(q, k, v, 0.5, True)
+        assert np.abs(out.numpy() - want_o[:, :, rows]).max() <= 1e-6
+        assert np.abs(lse.numpy() - want_l[:, :, rows]).max() <= 1e-5
+        # pass-Q decode inside the group, query sent from group rank 1
+        qd = q[:, :, :1].clone() if me == 1 else torch.zeros_like(q[:, :, :1])
+        od, ld = pass_q_decode(qd, part(k), part(v), 0.5, src=1, group=grp,
+                               transport=HostTransport(grp), blocks=OracleBlocks())
+        wo, wl = attention(q[:, :, :1], k, v, 0.5, False)
+        assert np.abs(od.numpy() - wo[:, :, 0]).max() <= 1e-6
+        assert np.abs(ld.numpy() - wl[:, :, 0]).max() <= 1e-5
+    except Exception:
+        errq.put((rank, traceback.format_exc()))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rings_on_process_subgroups():
+    world = 4
+    ctx = mp.get_context("spawn")
+    errq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_subgroup_main, args=(r, world, port, errq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    errs = []
+    while not errq.empty():
+        errs.append(errq.get())
+    assert not errs, errs
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
