@@ -330,3 +330,39 @@ def test_rings_on_process_subgroups():
         errs.append(errq.get())
     assert not errs, errs
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+
+
+def _dead_peer_main(rank, world, port, outq):
+    import time
+
+    import torch.distributed as dist
+
+    from ring_context_parallelism_ra_b200.distributed import HostTransport, ring_attention_forward
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        os._exit(0)          # leaves between steps: nothing of it is in flight
+    q = torch.zeros((1, 1, 4, 2), dtype=torch.float64)
+    t0 = time.time()
+    try:
+        ring_attention_forward(q, q, q, True, 1.0, transport=HostTransport(),
+                               blocks=OracleBlocks())
+        outq.put(("no error", time.time() - t0))
+    except Exception as e:  # noqa: BLE001
+        outq.put((type(e).__name__, time.time() - t0))
+    os._exit(0)
+
+
+def test_ring_reports_a_dead_peer_instead_of_hanging():
+    ctx = mp.get_context("spawn")
+    outq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dead_peer_main, args=(r, 2, port, outq)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode is not None for p in procs), "a rank hung"
+    kind, seconds = outq.get(timeout=5)
+    assert kind != "no error" and seconds < 60, (kind, seconds)
