@@ -351,6 +351,8 @@ def _dead_peer_main(rank, world, port, outq):
         outq.put(("no error", time.time() - t0))
     except Exception as e:  # noqa: BLE001
         outq.put((type(e).__name__, time.time() - t0))
+    outq.close()
+    outq.join_thread()       # the result must leave before the hard exit below
     os._exit(0)
 
 
