@@ -1,5 +1,9 @@
-"""Fused ring forward over a stream of host-resident batches, with the copies
-of one batch overlapped with the computation of its neighbours.
+"""Host-side drivers of the library's calls: the fused ring forward over a
+stream of host-resident batches (``RingForwardPipeline``), and a pass-Q
+decode step captured once as a CUDA graph (``PassQDecodeGraph``).
+
+RingForwardPipeline: the copies of one batch overlap the computation of its
+neighbours.
 
 Each batch goes host -> device (pinned memory, copy stream), through
 ``ra.ring_forward`` (compute stream) and its output and LSE back to pinned
@@ -14,7 +18,7 @@ import torch
 
 from . import ra
 
-__all__ = ["RingForwardPipeline"]
+__all__ = ["RingForwardPipeline", "PassQDecodeGraph"]
 
 
 class RingForwardPipeline:
@@ -82,3 +86,50 @@ class RingForwardPipeline:
         for s in range(self.depth):
             if self.used[s]:
                 stream.wait_event(self.out_done[s])
+
+
+class PassQDecodeGraph:
+    """Pass-Q decode over a fixed KV cache, captured once as a CUDA graph.
+
+    A decode step is P shard partials and their merge: with a short cache
+    every launch is short, and the CP study (page "上下文并行 (CP) 收益评估实验
+    设计", decode section) calls this step latency-bound.  Replaying the
+    captured graph enqueues the whole step at once.  Write the new query
+    token into ``q`` (a static device buffer [B, Hq, 1, d]) before each
+    ``replay``; the cache tensors must stay at their addresses.  ``out`` and
+    ``lse`` hold the result after the replay has run on the stream.
+    """
+
+    def __init__(self, k, v, P, Hq, scale=None, stream=None):
+        B, Hkv, S, d = k.shape
+        if S % P:
+            raise ValueError("cache length must split into P equal shards")
+        dev = k.device
+        self.k, self.v, self.P, self.scale = k, v, P, scale
+        self.q = torch.zeros((B, Hq, 1, d), device=dev, dtype=k.dtype)
+        self.bufs = {
+            "o_parts": torch.empty((P, B, Hq, v.shape[-1]), device=dev, dtype=torch.float32),
+            "lse_parts": torch.empty((P, B, Hq), device=dev, dtype=torch.float32),
+            "workspace": torch.empty(ra.decode_workspace_bytes(B, Hq, Hkv, S // P),
+                                     dtype=torch.uint8, device=dev),
+            "out": torch.empty((B, Hq, v.shape[-1]), device=dev, dtype=k.dtype),
+            "lse": torch.empty((B, Hq), device=dev, dtype=torch.float32),
+        }
+        self.out, self.lse = self.bufs["out"], self.bufs["lse"]
+        self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
+        # one eager run first: the library sets up its per-device state
+        # (status word, kernel attributes) outside the capture
+        with torch.cuda.stream(self.stream):
+            self._step()
+        self.stream.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            self._step()
+
+    def _step(self):
+        ra.decode_pass_q(self.q, self.k, self.v, self.P, self.scale, self.bufs)
+
+    def replay(self):
+        """Enqueue one decode step; returns (out [B, Hq, d_v], lse [B, Hq])."""
+        self.graph.replay()
+        return self.out, self.lse

@@ -288,3 +288,19 @@ def test_host_pipeline_equals_direct_calls():
     o_last, l_last = pipe.wait((len(batches) - 1) % pipe.depth)
     want_o, want_l = ra.ring_forward(*(x.to(DEV) for x in batches[-1]), 4, True)
     assert torch.equal(o_last, want_o.cpu()) and torch.equal(l_last, want_l.cpu())
+
+
+def test_pass_q_decode_graph_replays_match_oracle():
+    # one captured decode step replayed for two different query tokens
+    from ring_context_parallelism_ra_b200.host_pipeline import PassQDecodeGraph
+    B, Hq, Hkv, S, d, P = 2, 16, 2, 8192, 128, 4
+    _, k, v = make_qkv(B, Hq, Hkv, 1, S, d, d, torch.bfloat16, seed=81)
+    graph = PassQDecodeGraph(k.to(DEV), v.to(DEV), P, Hq)
+    for seed in (82, 83):
+        q, _, _ = make_qkv(B, Hq, Hkv, 1, 1, d, d, torch.bfloat16, seed=seed)
+        graph.q.copy_(q.to(DEV))
+        out, lse = graph.replay()
+        torch.cuda.synchronize()
+        want_o, want_l = oracle_attention(q, k, v, 1.0 / math.sqrt(d), False)
+        check_out(out, want_o[:, :, 0], "bf16")
+        check_lse(lse, want_l[:, :, 0])
