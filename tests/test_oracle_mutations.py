@@ -278,3 +278,75 @@ def test_blockwise_pins_catch_planted_mistake(name):
     old, new = BLOCKWISE_MUTANTS[name]
     mod = _mutant("blockwise", old, new)
     assert not all(_holds(p, mod) for p in BLOCKWISE_PINS), name
+
+
+# ----------------------------------------------- blockwise backward forms --
+
+def _pin_ring_backward_equals_whole(mod):
+    from oracle.backward import attention_backward     # the unmodified oracle
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((1, 4, 12, 3))
+    k = rng.standard_normal((1, 2, 12, 3))
+    v = rng.standard_normal((1, 2, 12, 2))
+    g = rng.standard_normal((1, 4, 12, 2))
+    for causal in (True, False):
+        want = attention_backward(q, k, v, g, 0.6, causal)
+        for P in (1, 2, 3, 4):
+            got = mod.ring_attention_backward(q, k, v, g, 0.6, causal, P)
+            for a, b in zip(got, want):
+                assert np.abs(a - b).max() <= 1e-12
+
+
+def _pin_block_shares_sum_to_whole(mod):
+    from oracle.attention import attention
+    from oracle.backward import attention_backward, row_delta
+    rng = np.random.default_rng(13)
+    n, P = 12, 3
+    q = rng.standard_normal((1, 2, n, 3))
+    k = rng.standard_normal((1, 1, n, 3))
+    v = rng.standard_normal((1, 1, n, 2))
+    g = rng.standard_normal((1, 2, n, 2))
+    o, lse = attention(q, k, v, 0.5, True)
+    d = row_delta(o, g)
+    dq, dk, dv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    L = n // P
+    pos = np.arange(n)
+    for i in range(P):
+        r = slice(i * L, (i + 1) * L)
+        for j in range(P):
+            c = slice(j * L, (j + 1) * L)
+            a, b, e = mod.block_backward_share(q[:, :, r], k[:, :, c], v[:, :, c], g[:, :, r],
+                                               lse[:, :, r], d[:, :, r], 0.5, True, pos[r], pos[c])
+            dq[:, :, r] += a
+            dk[:, :, c] += b
+            dv[:, :, c] += e
+    for x, w in zip((dq, dk, dv), attention_backward(q, k, v, g, 0.5, True)):
+        assert np.abs(x - w).max() <= 1e-12
+
+
+BLOCK_BACKWARD_PINS = [_pin_ring_backward_equals_whole, _pin_block_shares_sum_to_whole]
+
+BLOCK_BACKWARD_MUTANTS = {
+    "dK share delivered to the query partition": (
+        "dk[b, g, k0:k1] += scale * (ds.T @ qh[q0:q1])", "dk[b, g, q0:q1] += scale * (ds.T @ qh[q0:q1])"),
+    "block-local softmax instead of the final LSE": (
+        "p[live] = np.exp(s[live] - lse_i[live, None])",
+        "p[live] = np.exp(s[live] - s[live].max(axis=1, keepdims=True))"),
+    "diagonal blocks skipped": ("if not vis.any():", "if not vis.all():"),
+    "D of the key rows": ("ds = p * (dp - dlt[b, h, q0:q1, None])", "ds = p * (dp - dlt[b, h, k0:k1, None])"),
+    "block share without D": ("ds = p * (doh @ vv.T - delta[b, h][:, None])", "ds = p * (doh @ vv.T)"),
+    "block share mask off by one": ("s = np.where(kp[None, :] <= qp[:, None], s, -np.inf)",
+                                    "s = np.where(kp[None, :] < qp[:, None], s, -np.inf)"),
+}
+
+
+def test_block_backward_pins_hold_for_the_oracle():
+    import oracle.backward as mod
+    assert all(_holds(p, mod) for p in BLOCK_BACKWARD_PINS)
+
+
+@pytest.mark.parametrize("name", sorted(BLOCK_BACKWARD_MUTANTS))
+def test_block_backward_pins_catch_planted_mistake(name):
+    old, new = BLOCK_BACKWARD_MUTANTS[name]
+    mod = _mutant("backward", old, new)
+    assert not all(_holds(p, mod) for p in BLOCK_BACKWARD_PINS), name
