@@ -350,3 +350,78 @@ def test_block_backward_pins_catch_planted_mistake(name):
     old, new = BLOCK_BACKWARD_MUTANTS[name]
     mod = _mutant("backward", old, new)
     assert not all(_holds(p, mod) for p in BLOCK_BACKWARD_PINS), name
+
+
+# ------------------------------------------------- classification, costs --
+
+def _pin_class_matches_mask(mod):
+    from oracle.block_class import block_class_bruteforce   # the unmodified rule
+    for n, bq, bk in ((37, 8, 5), (64, 16, 16), (20, 3, 4)):
+        for qo, ko in ((0, 0), (5, 0), (0, 9)):
+            for causal in (True, False):
+                a = mod.block_class(n, n, bq, bk, qo, ko, causal)
+                b = block_class_bruteforce(n, n, bq, bk, qo, ko, causal)
+                assert np.array_equal(a, b)
+
+
+def _pin_partition_counts(mod):
+    m = mod.partition_class(8192, 4)
+    assert [(m == c).sum() for c in (0, 1, 2)] == [6, 4, 6]
+
+
+CLASS_PINS = [_pin_class_matches_mask, _pin_partition_counts]
+
+CLASS_MUTANTS = {
+    "visible count off by one": ("vis = np.clip(q_pos - (k_offset + k_start) + 1, 0, k_len)",
+                                 "vis = np.clip(q_pos - (k_offset + k_start), 0, k_len)"),
+    "FULL when any row sees the whole tile": ("if (r == k_len).all():", "if (r == k_len).any():"),
+    "query positions from the key offset": ("q_pos = q_offset + np.arange", "q_pos = k_offset + np.arange"),
+}
+
+
+def test_class_pins_hold_for_the_oracle():
+    import oracle.block_class as mod
+    assert all(_holds(p, mod) for p in CLASS_PINS)
+
+
+@pytest.mark.parametrize("name", sorted(CLASS_MUTANTS))
+def test_class_pins_catch_planted_mistake(name):
+    old, new = CLASS_MUTANTS[name]
+    assert not all(_holds(p, _mutant("block_class", old, new)) for p in CLASS_PINS), name
+
+
+def _pin_flops_count_pairs(mod):
+    for n, dqk, dv, H in ((16, 8, 4, 2), (12, 192, 128, 3)):
+        pairs = n * n
+        assert mod.prefill_flops(1, n, dqk, dv, H, causal=False) == 2 * pairs * (dqk + dv) * H
+        assert mod.prefill_flops(1, n, dqk, dv, H, causal=True) == pairs * (dqk + dv) * H
+
+
+def _pin_kv_table_and_ring_bytes(mod):
+    import json
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "kv_cache_sizes.json")))
+    for row in g["rows"]:
+        assert mod.kv_cache_bytes(g["L"], g["h_kv"], g["d_h"], row["n"], g["b"]) / 2**30 == row["gib"]
+    assert mod.pass_kv_bytes_per_chip(1, 1000, 1152) == 0          # one chip sends nothing
+
+
+COST_PINS = [_pin_flops_count_pairs, _pin_kv_table_and_ring_bytes]
+
+COST_MUTANTS = {
+    "heads not counted": ("f = 2 * B * S * S * (d_qk + d_v) * heads", "f = 2 * B * S * S * (d_qk + d_v)"),
+    "causal not halved": ("return f // 2 if causal else f\n\n\ndef backward_flops",
+                          "return f\n\n\ndef backward_flops"),
+    "K or V missing from the cache": ("return 2 * L * h_kv * d_h * n * b", "return L * h_kv * d_h * n * b"),
+    "ring bytes without the (cp - 1) / cp factor": ("return (cp - 1) * S * c_kv / cp", "return S * c_kv / cp"),
+}
+
+
+def test_cost_pins_hold_for_the_oracle():
+    import oracle.costs as mod
+    assert all(_holds(p, mod) for p in COST_PINS)
+
+
+@pytest.mark.parametrize("name", sorted(COST_MUTANTS))
+def test_cost_pins_catch_planted_mistake(name):
+    old, new = COST_MUTANTS[name]
+    assert not all(_holds(p, _mutant("costs", old, new)) for p in COST_PINS), name
