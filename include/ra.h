@@ -184,6 +184,29 @@ int ra_decode_partial(const void* q, const void* k_shard, const void* v_shard,
                       void* stream);
 
 /*
+ * ra_decode_partials -- the P shard partials of pass-Q decode at once, for a
+ * cache that one device holds whole: the same partials as P calls of
+ * ra_decode_partial (one per token range of n_k / P tokens), computed by one
+ * launch over every chunk of every shard and one merge of each shard's
+ * chunks.  With short shards the P separate launches leave SMs idle; this
+ * call keeps them busy.  ra_decode_merge then combines the partials.
+ *   q           : device bf16 [B, Hq, 1, d_qk].
+ *   k, v        : device bf16 [B, Hkv, n_k, d] (the whole cache, dense).
+ *   P           : shards; n_k % P == 0, and (n_k / P) % 2048 == 0 when P > 1
+ *                 (whole 2048-token chunks per shard), else RA_ERR_UNSUPPORTED.
+ *   shape       : n_q must be 1; n_k = the whole cache; d_qk == d_v == 128.
+ *   o_parts     : device fp32 [P, B, Hq, d_v], each normalised over its shard.
+ *   lse_parts   : device fp32 [P, B, Hq].
+ *   workspace   : device, >= ra_decode_workspace_bytes(shape) with n_k the
+ *                 whole cache, 16-B aligned, caller-owned.
+ * Errors: RA_ERR_INVALID, RA_ERR_UNSUPPORTED (dims, dtype, shard length),
+ * RA_ERR_CUDA.
+ */
+int ra_decode_partials(const void* q, const void* k, const void* v, int P, const ra_shape* shape,
+                       float scale, float* o_parts, float* lse_parts, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
  * ra_decode_partial_noalloc -- ra_decode_partial without a caller workspace.
  * The pages have no counterpart of this call; it exists for callers that
  * cannot allocate device memory: a plugin inside a host runtime that owns all

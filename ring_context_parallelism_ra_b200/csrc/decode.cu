@@ -76,7 +76,13 @@ struct DecodeArgs {
   const __nv_bfloat16* q;
   int B, Hq, Hkv, G, n_k;
   int n_chunks;
+  int shards;     // the cache is this many equal shards of whole chunks
   float scale_log2;
+  // Chunk ch is chunk c = ch % (n_chunks / shards) of shard p = ch / (n_chunks
+  // / shards); its partial is row (c * shards + p) * B*Hq + (b*Hq + h), so the
+  // chunks of one position c across all shards are consecutive and one LSE
+  // merge over the n_chunks / shards positions leaves the shards' partials
+  // stacked [shards][B*Hq].  shards = 1: row ch * B*Hq + (b*Hq + h).
   float* ws_o;    // [n_chunks][B*Hq][kD]
   float* ws_lse;  // [n_chunks][B*Hq]
   DevCtx ctx;
@@ -286,8 +292,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_chunk_kernel(
             L += f[w] * comb_ml[(w * 16 + row) * 2 + 1];
           }
           const float inv = L > 0.f ? 1.f / L : 0.f;
-          const long long orow = static_cast<long long>(ch) * a.B * a.Hq +
-                                 static_cast<long long>(b) * a.Hq + g * a.G + row;
+          const int cps = a.n_chunks / a.shards;
+          const long long slot = static_cast<long long>(ch % cps) * a.shards + ch / cps;
+          const long long orow = slot * a.B * a.Hq + static_cast<long long>(b) * a.Hq +
+                                 g * a.G + row;
           float* dst = a.ws_o + orow * kD + c0;
 #pragma unroll
           for (int c = 0; c < 16; c += 4) {
@@ -332,8 +340,12 @@ size_t decode_workspace_bytes(const ra_shape& s) {
 
 int launch_decode_partial(const void* q, const void* k, const void* v, long long kv_head_stride,
                           const ra_shape& s, float scale, float* o_part, float* lse_part,
-                          float* workspace, const DeviceInfo& dev, cudaStream_t stream) {
+                          float* workspace, const DeviceInfo& dev, cudaStream_t stream,
+                          int shards) {
   if (s.d_qk != kD || s.d_v != kD || s.dtype != RA_BF16 || s.Hq / s.Hkv > 16)
+    return RA_ERR_UNSUPPORTED;
+  // several shards need whole chunks in every shard
+  if (shards < 1 || (shards > 1 && (s.n_k % shards != 0 || (s.n_k / shards) % kChunk != 0)))
     return RA_ERR_UNSUPPORTED;
   CUtensorMap tk, tv;
   const uint64_t heads = static_cast<uint64_t>(s.B) * s.Hkv;
@@ -349,6 +361,7 @@ int launch_decode_partial(const void* q, const void* k, const void* v, long long
   a.G = s.Hq / s.Hkv;
   a.n_k = s.n_k;
   a.n_chunks = (s.n_k + kChunk - 1) / kChunk;
+  a.shards = shards;
   a.scale_log2 = scale * kLog2e;
   const long long rows = static_cast<long long>(s.B) * s.Hq;
   a.ws_o = workspace;
@@ -362,8 +375,9 @@ int launch_decode_partial(const void* q, const void* k, const void* v, long long
   decode_chunk_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tk, tv, a);
   note_launch();
   if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
-  return launch_lse_merge(a.ws_o, a.ws_lse, a.n_chunks, rows, kD, o_part, RA_F32, lse_part,
-                          dev.num_sms, stream);
+  // o_part / lse_part: [shards][B*Hq](kD): one partial per shard
+  return launch_lse_merge(a.ws_o, a.ws_lse, a.n_chunks / shards, rows * shards, kD, o_part,
+                          RA_F32, lse_part, dev.num_sms, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -45,7 +45,7 @@ int launch_tc_attention(const void* q, const void* k, const void* v, const ra_sh
 size_t decode_workspace_bytes(const ra_shape& s);
 int launch_decode_partial(const void* q, const void* k, const void* v, long long kv_head_stride,
                           const ra_shape& s, float scale, float* o_part, float* lse_part,
-                          float* workspace, const DeviceInfo& dev, cudaStream_t stream);
+                          float* workspace, const DeviceInfo& dev, cudaStream_t stream, int shards = 1);
 
 // Same without a caller workspace: the chunk partials go to a file-scope
 // device array of decode_static_scratch_bytes() bytes.

@@ -271,6 +271,28 @@ int ra_decode_partial(const void* q, const void* k_shard, const void* v_shard,
                                static_cast<cudaStream_t>(stream));
 }
 
+int ra_decode_partials(const void* q, const void* k, const void* v, int P,
+                       const ra_shape* shape, float scale, float* o_parts, float* lse_parts,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_common(shape);
+  if (rc != RA_OK) return rc;
+  if (!q || !k || !v || !o_parts || !lse_parts || !workspace) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_parts) ||
+      !aligned16(lse_parts) || !aligned16(workspace))
+    return RA_ERR_INVALID;
+  if (shape->n_q != 1 || P < 1 || shape->n_k % P != 0) return RA_ERR_INVALID;
+  if (shape->dtype != RA_BF16 || shape->d_qk != 128 || shape->d_v != 128 ||
+      shape->Hq / shape->Hkv > 16 || (P > 1 && (shape->n_k / P) % 2048 != 0))
+    return RA_ERR_UNSUPPORTED;
+  if (workspace_bytes < decode_workspace_bytes(*shape)) return RA_ERR_INVALID;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc != RA_OK) return rc;
+  return launch_decode_partial(q, k, v, shape->n_k, *shape, scale, o_parts, lse_parts,
+                               static_cast<float*>(workspace), dev,
+                               static_cast<cudaStream_t>(stream), P);
+}
+
 int ra_decode_partial_noalloc(const void* q, const void* k_shard, const void* v_shard,
                               long long kv_head_stride, const ra_shape* shape, float scale,
                               float* o_part, float* lse_part, void* stream) {

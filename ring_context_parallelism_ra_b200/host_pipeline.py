@@ -110,7 +110,7 @@ class PassQDecodeGraph:
         self.bufs = {
             "o_parts": torch.empty((P, B, Hq, v.shape[-1]), device=dev, dtype=torch.float32),
             "lse_parts": torch.empty((P, B, Hq), device=dev, dtype=torch.float32),
-            "workspace": torch.empty(ra.decode_workspace_bytes(B, Hq, Hkv, S // P),
+            "workspace": torch.empty(ra.decode_workspace_bytes(B, Hq, Hkv, S),
                                      dtype=torch.uint8, device=dev),
             "out": torch.empty((B, Hq, v.shape[-1]), device=dev, dtype=k.dtype),
             "lse": torch.empty((B, Hq), device=dev, dtype=torch.float32),

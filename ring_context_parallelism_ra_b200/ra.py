@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "RAError", "library_path", "lib", "Shape", "block_partial", "block_partial_strided",
     "lse_merge", "ring_forward", "ring_forward_striped",
-    "ring_forward_host", "decode_workspace_bytes", "decode_partial", "decode_partial_noalloc",
+    "ring_forward_host", "decode_workspace_bytes", "decode_partial", "decode_partials",
+    "decode_partial_noalloc",
     "decode_merge",
     "decode_pass_q", "backward_workspace_bytes", "backward_delta", "ring_backward",
     "ring_backward_striped", "block_backward",
@@ -34,7 +35,7 @@ RA_F32, RA_BF16 = 0, 1
 EXPORTED = (
     "ra_block_partial", "ra_block_partial_strided", "ra_lse_merge", "ra_ring_forward",
     "ra_ring_forward_striped", "ra_decode_workspace_bytes",
-    "ra_decode_partial", "ra_decode_partial_noalloc", "ra_decode_merge",
+    "ra_decode_partial", "ra_decode_partials", "ra_decode_partial_noalloc", "ra_decode_merge",
     "ra_backward_workspace_bytes", "ra_backward_delta", "ra_ring_backward",
     "ra_ring_backward_striped", "ra_block_backward", "ra_block_class", "ra_block_class_device",
     "ra_get_status", "ra_set_wait_limit_ns", "ra_check_wait_timeout", "ra_status_string",
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "ra_decode_workspace_bytes": (sz, [sp]),
             "ra_decode_partial": (i, [vp, vp, vp, ctypes.c_longlong, sp, f, vp, vp, vp, sz, vp]),
             "ra_decode_partial_noalloc": (i, [vp, vp, vp, ctypes.c_longlong, sp, f, vp, vp, vp]),
+            "ra_decode_partials": (i, [vp, vp, vp, i, sp, f, vp, vp, vp, sz, vp]),
             "ra_decode_merge": (i, [vp, vp, i, sp, vp, i, vp, vp]),
             "ra_backward_workspace_bytes": (sz, [sp]),
             "ra_backward_delta": (i, [vp, vp, sp, vp, vp]),
@@ -422,8 +424,40 @@ def decode_merge(o_parts, lse_parts, out_dtype=torch.bfloat16, out=None, lse=Non
     return o.view(B, H, d), l.view(B, H)
 
 
+def decode_partials(q, k, v, P, scale=None, workspace=None, o_parts=None, lse_parts=None,
+                    stream=None):
+    """The P shard partials of a [B, Hkv, S, d] cache in one launch (shards of
+    S / P tokens, whole 2048-token chunks).  Returns (O_parts [P,B,Hq,d],
+    LSE_parts [P,B,Hq])."""
+    B, Hq, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence")
+    _, Hkv, S, _ = k.shape
+    s = Shape(B, Hq, Hkv, 1, S, d, v.shape[-1], _dtype_code(q.dtype))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if workspace is None:
+        workspace = torch.empty(int(lib().ra_decode_workspace_bytes(ctypes.byref(s))),
+                                dtype=torch.uint8, device=q.device)
+    if o_parts is None:
+        o_parts = torch.empty((P, B, Hq, v.shape[-1]), device=q.device, dtype=torch.float32)
+    if lse_parts is None:
+        lse_parts = torch.empty((P, B, Hq), device=q.device, dtype=torch.float32)
+    _need(k, "k", q.dtype)
+    _need(v, "v", q.dtype)
+    rc = lib().ra_decode_partials(_need(q, "q"), _need(k, "k"), _need(v, "v"), P, ctypes.byref(s),
+                                  float(scale), _need(o_parts, "o_parts", torch.float32),
+                                  _need(lse_parts, "lse_parts", torch.float32),
+                                  ctypes.c_void_p(workspace.data_ptr()),
+                                  ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                  _stream(stream))
+    _check("ra_decode_partials", rc)
+    return o_parts, lse_parts
+
+
 def decode_pass_q(q, k, v, P, scale=None, bufs=None):
-    """Whole pass-Q decode on one GPU: P shard partials, then the merge."""
+    """Whole pass-Q decode on one GPU: P shard partials, then the merge.  With
+    shards of whole 2048-token chunks the partials come from one launch
+    (decode_partials); otherwise one decode_partial call per shard."""
     B, Hq, _, d = q.shape
     S = k.shape[2]
     if S % P:
@@ -437,8 +471,14 @@ def decode_pass_q(q, k, v, P, scale=None, bufs=None):
     if lse_parts is None:
         lse_parts = torch.empty((P, B, Hq), device=q.device, dtype=torch.float32)
     ws = bufs.get("workspace")
-    for p in range(P):
-        decode_partial(q, k, v, p * L, L, scale, ws, o_parts[p], lse_parts[p])
+    if P == 1 or L % 2048 == 0:
+        if ws is not None and ws.numel() < int(lib().ra_decode_workspace_bytes(
+                ctypes.byref(Shape(B, Hq, k.shape[1], 1, S, d, v.shape[-1], _dtype_code(q.dtype))))):
+            raise ValueError("workspace smaller than ra_decode_workspace_bytes of the whole cache")
+        decode_partials(q, k, v, P, scale, ws, o_parts, lse_parts)
+    else:
+        for p in range(P):
+            decode_partial(q, k, v, p * L, L, scale, ws, o_parts[p], lse_parts[p])
     return decode_merge(o_parts, lse_parts, q.dtype, bufs.get("out"), bufs.get("lse"))
 
 

@@ -94,6 +94,12 @@ def test_validation_rejects_bad_arguments_before_launch():
     sd3 = _shape(n_q=1, Hq=8, Hkv=1, n_k=4096, d_qk=64, d_v=64)
     assert L.ra_decode_partial(p, p, p, 4096, ctypes.byref(sd3), 1.0, p, p, p, 1 << 30, nul) == UNS
     assert L.ra_decode_merge(p, p, 2, ctypes.byref(_shape(n_q=4)), p, 0, p, nul) == INV
+    # shards in one launch need whole 2048-token chunks per shard
+    sp = _shape(n_q=1, Hq=8, Hkv=1, n_k=6000)
+    assert L.ra_decode_partials(p, p, p, 3, ctypes.byref(sp), 1.0, p, p, p, 1 << 30, nul) == UNS
+    assert L.ra_decode_partials(p, p, p, 7, ctypes.byref(sp), 1.0, p, p, p, 1 << 30, nul) == INV
+    sp2 = _shape(n_q=1, Hq=8, Hkv=1, n_k=8192)
+    assert L.ra_decode_partials(p, p, p, 4, ctypes.byref(sp2), 1.0, p, p, p, 16, nul) == INV  # ws
     # empty inputs are rejected, not launched: no sequence, no batch, no heads
     s0 = _shape(n_q=0, n_k=0)
     assert L.ra_ring_forward(p, p, p, 1, 1, 1.0, p, p, ctypes.byref(s0), nul) == INV

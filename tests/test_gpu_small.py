@@ -250,6 +250,26 @@ def test_decode_pass_q_matches_oracle(case):
     check_lse(lse, want_l[:, :, 0])
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,S,P", [(2, 16, 2, 16384, 4), (1, 8, 1, 8192, 2),
+                                         (4, 64, 8, 32768, 8), (1, 8, 2, 6144, 3)])
+def test_decode_partials_one_launch_match_per_shard_oracle(B, Hq, Hkv, S, P):
+    # every shard's partial from one launch, then the shard merge
+    q, k, v = make_qkv(B, Hq, Hkv, 1, S, 128, 128, torch.bfloat16, seed=S + P)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    scale = 1 / math.sqrt(128)
+    L = S // P
+    o_parts, l_parts = ra.decode_partials(qd, kd, vd, P, scale)
+    for p in range(P):
+        wo, wl_ = oracle_attention(q, k[:, :, p * L:(p + 1) * L], v[:, :, p * L:(p + 1) * L],
+                                   scale, False)
+        check_out(o_parts[p], wo[:, :, 0], "bf16", f"shard {p} O")
+        check_lse(l_parts[p], wl_[:, :, 0], f"shard {p} LSE")
+    out, lse = ra.decode_pass_q(qd, kd, vd, P, scale)
+    want_o, want_l = oracle_attention(q, k, v, scale, False)
+    check_out(out, want_o[:, :, 0], "bf16")
+    check_lse(lse, want_l[:, :, 0])
+
+
 # ------------------------------------------------------------- failure ----
 
 def test_bounded_wait_reports_timeout_and_context_survives():
