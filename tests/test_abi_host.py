@@ -199,3 +199,10 @@ def test_missing_library_fails_loudly(tmp_path):
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "is missing" in r.stdout
+
+
+def test_decode_graph_rejects_uneven_shards_before_any_gpu_work():
+    from ring_context_parallelism_ra_b200.host_pipeline import PassQDecodeGraph
+    k = torch.zeros((1, 1, 1000, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="equal shards"):
+        PassQDecodeGraph(k, k, 3, 8)
