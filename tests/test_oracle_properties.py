@@ -81,3 +81,48 @@ def test_ring_equals_definition_for_any_partition_count(P, L, grp, causal, seed,
 def test_tile_class_equals_mask(nq, nk, bq, bk, qo, ko, causal):
     assert np.array_equal(block_class(nq, nk, bq, bk, qo, ko, causal),
                           block_class_bruteforce(nq, nk, bq, bk, qo, ko, causal))
+
+
+@SETTINGS
+@given(P=st.integers(1, 5), L=st.integers(1, 4), grp=st.integers(1, 2), causal=st.booleans(),
+       seed=st.integers(0, 2**31 - 1))
+def test_ring_backward_equals_whole_rows(P, L, grp, causal, seed):
+    from oracle.backward import attention_backward, ring_attention_backward
+    rng = np.random.default_rng(seed)
+    n = P * L
+    q = rng.standard_normal((1, 2 * grp, n, 3))
+    k = rng.standard_normal((1, 2, n, 3))
+    v = rng.standard_normal((1, 2, n, 2))
+    g = rng.standard_normal((1, 2 * grp, n, 2))
+    order = [list(rng.permutation(P)) for _ in range(P)]
+    got = ring_attention_backward(q, k, v, g, 0.5, causal, P, order=lambda P_, i: order[i])
+    for a, b in zip(got, attention_backward(q, k, v, g, 0.5, causal)):
+        assert np.abs(a - b).max() <= 1e-12
+
+
+@SETTINGS
+@given(nq=st.integers(2, 6), nk=st.integers(2, 6), grp=st.integers(1, 2), causal=st.booleans(),
+       qo=st.integers(0, 4), seed=st.integers(0, 2**31 - 1))
+def test_backward_equals_autodiff(nq, nk, grp, causal, qo, seed):
+    import torch
+
+    from oracle.backward import attention_backward
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, 2 * grp, nq, 3))
+    k = rng.standard_normal((1, 2, nk, 3))
+    v = rng.standard_normal((1, 2, nk, 2))
+    g = rng.standard_normal((1, 2 * grp, nq, 2))
+    qpos, kpos = qo + np.arange(nq), np.arange(nk)
+    if causal and (kpos[0] > qpos).any():
+        return            # rows that see no key have no softmax to differentiate
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    kk = tk.repeat_interleave(grp, dim=1)
+    vv = tv.repeat_interleave(grp, dim=1)
+    s = torch.einsum("bhtc,bhuc->bhtu", tq, kk) * 0.9
+    if causal:
+        s = s.masked_fill(torch.tensor(kpos[None, :] > qpos[:, None]), float("-inf"))
+    o = torch.einsum("bhtu,bhuc->bhtc", torch.softmax(s, dim=-1), vv)
+    (o * torch.tensor(g)).sum().backward()
+    got = attention_backward(q, k, v, g, 0.9, causal, q_offset=qo)
+    for a, t in zip(got, (tq, tk, tv)):
+        assert np.abs(a - t.grad.numpy()).max() <= 1e-12
