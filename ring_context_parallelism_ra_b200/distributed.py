@@ -204,6 +204,15 @@ def partition_positions(rank: int, P: int, L: int, striped: bool):
     return (rank, P) if striped else (rank * L, 1)
 
 
+def _ring_check(q, k, v):
+    """The ring assumes one equal partition per rank: Q, K and V of a rank
+    hold the same tokens."""
+    if not (q.shape[2] == k.shape[2] == v.shape[2]) or q.shape[0] != k.shape[0] or \
+            k.shape[:3] != v.shape[:3] or q.shape[-1] != k.shape[-1] or q.shape[1] % k.shape[1]:
+        raise ValueError(f"ring partitions disagree: q {tuple(q.shape)}, k {tuple(k.shape)}, "
+                         f"v {tuple(v.shape)}")
+
+
 def _ring(group):
     P = dist.get_world_size(group)
     i = dist.get_rank(group)
@@ -215,6 +224,7 @@ def ring_attention_forward(q, k, v, causal=True, scale=None, striped=False, grou
     """This rank's output (O_i [B, Hq, L, d_v] in q's dtype, LSE_i fp32
     [B, Hq, L]) of exact attention over the whole sequence, its query
     partition meeting every KV partition as they pass around the ring."""
+    _ring_check(q, k, v)
     P, i, nxt, prv = _ring(group)
     transport = transport or default_transport(group)
     blocks = blocks or KernelBlocks()
@@ -245,6 +255,9 @@ def ring_attention_backward(q, k, v, out, lse, dout, causal=True, scale=None, st
                             group=None, transport=None, blocks=None):
     """This rank's gradients (dQ_i, dK_i, dV_i, in q's dtype) of
     ``ring_attention_forward``; ``out`` and ``lse`` are its outputs here."""
+    _ring_check(q, k, v)
+    if out.shape[:3] != q.shape[:3] or dout.shape != out.shape or lse.shape != q.shape[:3]:
+        raise ValueError("out, lse and dout must match this rank's query partition")
     P, i, nxt, prv = _ring(group)
     transport = transport or default_transport(group)
     blocks = blocks or KernelBlocks()

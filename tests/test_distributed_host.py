@@ -168,7 +168,8 @@ def _ulysses_main(rank, world, port, errq):
 
     from oracle.attention import attention
     from oracle.backward import attention_backward
-    from ring_context_parallelism_ra_b200.distributed import (HostTransport,
+    from ring_context_parallelism_ra_b200.distributed import (HostTransport, pass_q_decode,
+                                                              ring_attention_forward,
                                                               ulysses_attention_backward,
                                                               ulysses_attention_forward)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -197,6 +198,19 @@ def _ulysses_main(rank, world, port, errq):
         want = attention_backward(q, k, v, g, 0.4, True)
         for got, w in zip(grads, want):
             assert np.abs(got.numpy() - w[:, :, rows]).max() <= 1e-9
+        # argument errors are raised on every rank before any exchange
+        odd = torch.zeros((B, world + 1, L, d), dtype=torch.float64)
+        with pytest.raises(ValueError, match="divisible"):
+            ulysses_attention_forward(odd, odd, odd, True, 0.4, transport=tr, blocks=blocks)
+        with pytest.raises(ValueError, match="disagree"):
+            ring_attention_forward(part(q), part(k)[:, :, :-1], part(v), True, 0.4, transport=tr,
+                                   blocks=blocks)
+        with pytest.raises(ValueError, match="one query token"):
+            pass_q_decode(part(q), part(k), part(v), 0.4, transport=tr, blocks=blocks)
+        # the group is still in step: one more exchange completes
+        out2, _ = ulysses_attention_forward(part(q), part(k), part(v), True, 0.4,
+                                            transport=tr, blocks=blocks)
+        assert torch.equal(out2, out)
     except Exception:
         errq.put((rank, traceback.format_exc()))
         raise
