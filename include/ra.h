@@ -184,8 +184,10 @@ int ra_decode_partial(const void* q, const void* k_shard, const void* v_shard,
                       void* stream);
 
 /*
- * ra_decode_partials -- the P shard partials of pass-Q decode at once, for a
- * cache that one device holds whole: the same partials as P calls of
+ * ra_decode_partials -- the P shard partials of pass-Q decode (page "上下文并行
+ * (CP) 收益评估实验设计", decode section: each chip attends over its S/cp
+ * tokens) at once, for a cache that one device holds whole: the same
+ * partials as P calls of
  * ra_decode_partial (one per token range of n_k / P tokens), computed by one
  * launch over every chunk of every shard and one merge of each shard's
  * chunks.  With short shards the P separate launches leave SMs idle; this
