@@ -382,3 +382,42 @@ def test_ring_reports_a_dead_peer_instead_of_hanging():
     assert all(p.exitcode is not None for p in procs), "a rank hung"
     kind, seconds = outq.get(timeout=5)
     assert kind != "no error" and seconds < 60, (kind, seconds)
+
+
+def test_nccl_transport_addresses_global_ranks_of_a_subgroup(monkeypatch):
+    # NCCL needs GPUs; a recording stand-in for torch.distributed checks the
+    # calls the transport makes: peers and roots are global ranks of the group
+    import types
+
+    from ring_context_parallelism_ra_b200 import distributed as D
+
+    calls = []
+
+    def isend(*a, **k):
+        raise AssertionError("the transport batches its point-to-point calls")
+
+    def irecv(*a, **k):
+        raise AssertionError("the transport batches its point-to-point calls")
+
+    class P2POp:
+        def __init__(self, op, t, peer, group):
+            self.op, self.peer = ("send" if op is isend else "recv"), peer
+
+    fake = types.SimpleNamespace(
+        P2POp=P2POp, isend=isend, irecv=irecv,
+        batch_isend_irecv=lambda ops: calls.append(("batch", [(o.op, o.peer) for o in ops])) or [],
+        get_global_rank=lambda group, r: {0: 4, 1: 6, 2: 7}[r],   # group ranks -> global 4, 6, 7
+        broadcast=lambda t, src, group=None: calls.append(("broadcast", src)),
+        all_gather_into_tensor=lambda out, inp, group=None: calls.append(
+            ("all_gather", tuple(out.shape), tuple(inp.shape))),
+    )
+    monkeypatch.setattr(D, "dist", fake)
+    tr = D.NcclTransport(group="g")
+    tr.exchange([torch.zeros(2), torch.zeros(3)], [torch.zeros(2), torch.zeros(3)],
+                nxt=2, prv=1).wait()
+    tr.broadcast(torch.zeros(1), src=2)
+    tr.all_gather(torch.zeros(3, 5), torch.zeros(5))
+    assert [c[0] for c in calls] == ["batch", "broadcast", "all_gather"]
+    assert calls[0][1] == [("send", 7), ("send", 7), ("recv", 6), ("recv", 6)]
+    assert calls[1] == ("broadcast", 7)
+    assert calls[2] == ("all_gather", (3, 5), (5,))
