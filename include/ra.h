@@ -254,7 +254,10 @@ int ra_decode_merge(const float* o_parts, const float* lse_parts, int P, const r
  * with dK, dV of a KV head summed over the query heads of its group.  In the
  * ring, KV_j travels with its accumulators dK_j, dV_j and collects one share
  * per query partition while dQ_i collects at its partition.
- * Supported head dims (bf16 and fp32): d_qk, d_v in {64, 128}.
+ * Supported head dims: d_qk, d_v in {64, 128} (bf16 on tensor cores, fp32
+ * on the CUDA cores); bf16 d_qk = 192 with d_v in {64, 128} (the MLA-shaped
+ * head) on the exact-fp32 CUDA-core kernel, since its dK accumulator does not
+ * fit tensor memory beside S^T, dP^T and dV: correct, not fast.
  */
 
 /*

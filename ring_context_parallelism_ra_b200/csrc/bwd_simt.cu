@@ -1,6 +1,10 @@
-// Exact-fp32 backward pass for fp32 inputs (FMA pipes, no tensor cores):
-// the same gradients and the same walk as the tensor-core kernel (bwd.cuh),
-// with 64-key tiles against 64-row query tiles.
+// Exact-fp32 backward pass on the FMA pipes (no tensor cores): the same
+// gradients and the same walk as the tensor-core kernel (bwd.cuh), with
+// 64-key tiles against 64-row query tiles.  It serves fp32 inputs, and bf16
+// inputs whose d_qk = 192 leaves the tensor-core kernel no room in tensor
+// memory for the dK accumulator (inputs widened to fp32 on load; dK, dV
+// stored in the input dtype, or added into the caller's fp32 accumulators
+// for a block share).
 //
 // One CTA (256 threads) per key tile of one (batch, KV head).  Per visit the
 // CTA stages Q_t, dO_t and the rows' -LSE log2(e), D in shared memory, forms
@@ -27,11 +31,28 @@ struct SCfg {
   static constexpr int SMEM = SMEM_FLOATS * 4;
 };
 
-template <int DQK, int DV>
-__global__ void __launch_bounds__(kSimtThreads) bwd_simt_kernel(const float* __restrict__ q,
-                                                               const float* __restrict__ k,
-                                                               const float* __restrict__ v,
-                                                               const float* __restrict__ dout,
+__device__ __forceinline__ float widen(float x) { return x; }
+__device__ __forceinline__ float widen(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Store of a finished dK / dV entry: the input dtype for the ring, or added
+// into the fp32 accumulator of a block share.
+template <typename T>
+__device__ __forceinline__ void put(void* base, long long i, float x, int block_mode) {
+  if (block_mode) {
+    float* p = static_cast<float*>(base) + i;
+    *p += x;
+  } else if constexpr (sizeof(T) == 4) {
+    static_cast<float*>(base)[i] = x;
+  } else {
+    static_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(x);
+  }
+}
+
+template <typename T, int DQK, int DV>
+__global__ void __launch_bounds__(kSimtThreads) bwd_simt_kernel(const T* __restrict__ q,
+                                                               const T* __restrict__ k,
+                                                               const T* __restrict__ v,
+                                                               const T* __restrict__ dout,
                                                                BwdArgs a) {
   using C = SCfg<DQK, DV>;
   extern __shared__ float sf[];
@@ -50,15 +71,15 @@ __global__ void __launch_bounds__(kSimtThreads) bwd_simt_kernel(const float* __r
   const int ty = tid >> 4, tx = tid & 15;
   const int ku = tid >> 2, kc = tid & 3;
 
-  const float* kb = k + (static_cast<long long>(it.bkv) * a.n_k + it.k0) * DQK;
-  const float* vb = v + (static_cast<long long>(it.bkv) * a.n_k + it.k0) * DV;
+  const T* kb = k + (static_cast<long long>(it.bkv) * a.n_k + it.k0) * DQK;
+  const T* vb = v + (static_cast<long long>(it.bkv) * a.n_k + it.k0) * DV;
   for (int i = tid; i < kBT * DQK; i += kSimtThreads) {
     const int r = i / DQK, c = i % DQK;
-    sK[r * C::KP + c] = r < it.klen ? kb[i] : 0.f;
+    sK[r * C::KP + c] = r < it.klen ? widen(kb[i]) : 0.f;
   }
   for (int i = tid; i < kBT * DV; i += kSimtThreads) {
     const int r = i / DV, c = i % DV;
-    sV[r * C::VP + c] = r < it.klen ? vb[i] : 0.f;
+    sV[r * C::VP + c] = r < it.klen ? widen(vb[i]) : 0.f;
   }
 
   float dk[DQK / 4], dv[DV / 4];
@@ -74,15 +95,15 @@ __global__ void __launch_bounds__(kSimtThreads) bwd_simt_kernel(const float* __r
     const int bh = it.b * a.Hq + h;
     const int q0 = qt * kBT;
     __syncthreads();  // previous visit done with the staged tiles
-    const float* qb = q + (static_cast<long long>(bh) * a.n_q + q0) * DQK;
-    const float* gb = dout + (static_cast<long long>(bh) * a.n_q + q0) * DV;
+    const T* qb = q + (static_cast<long long>(bh) * a.n_q + q0) * DQK;
+    const T* gb = dout + (static_cast<long long>(bh) * a.n_q + q0) * DV;
     for (int i = tid; i < kBT * DQK; i += kSimtThreads) {
       const int r = i / DQK, c = i % DQK;
-      sQ[r * C::KP + c] = r < w.qlen ? qb[i] : 0.f;
+      sQ[r * C::KP + c] = r < w.qlen ? widen(qb[i]) : 0.f;
     }
     for (int i = tid; i < kBT * DV; i += kSimtThreads) {
       const int r = i / DV, c = i % DV;
-      sdO[r * C::VP + c] = r < w.qlen ? gb[i] : 0.f;
+      sdO[r * C::VP + c] = r < w.qlen ? widen(gb[i]) : 0.f;
     }
     if (tid < kBT) {
       const long long vr = static_cast<long long>(bh) * a.ntq_ws * kBwdTile + q0 + tid;
@@ -142,27 +163,23 @@ __global__ void __launch_bounds__(kSimtThreads) bwd_simt_kernel(const float* __r
   }
   if (ku < it.klen) {
     const long long krow = static_cast<long long>(it.bkv) * a.n_k + it.k0 + ku;
-    float* dkp = static_cast<float*>(a.dk) + krow * DQK;
-    float* dvp = static_cast<float*>(a.dv) + krow * DV;
 #pragma unroll
-    for (int c = 0; c < DQK / 4; ++c) {
-      const float x = dk[c] * a.scale;
-      dkp[kc + 4 * c] = a.block_mode ? dkp[kc + 4 * c] + x : x;
-    }
+    for (int c = 0; c < DQK / 4; ++c) put<T>(a.dk, krow * DQK + kc + 4 * c, dk[c] * a.scale, a.block_mode);
 #pragma unroll
-    for (int c = 0; c < DV / 4; ++c)
-      dvp[kc + 4 * c] = a.block_mode ? dvp[kc + 4 * c] + dv[c] : dv[c];
+    for (int c = 0; c < DV / 4; ++c) put<T>(a.dv, krow * DV + kc + 4 * c, dv[c], a.block_mode);
   }
 }
 
-template <int DQK, int DV>
-int launch_simt_bwd_typed(const float* q, const float* k, const float* v, const float* dout,
+template <typename T, int DQK, int DV>
+int launch_simt_bwd_typed(const void* q, const void* k, const void* v, const void* dout,
                           const BwdArgs& a, cudaStream_t st) {
-  auto kern = bwd_simt_kernel<DQK, DV>;
+  auto kern = bwd_simt_kernel<T, DQK, DV>;
   constexpr int smem = SCfg<DQK, DV>::SMEM;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return RA_ERR_CUDA;
-  kern<<<a.items, kSimtThreads, smem, st>>>(q, k, v, dout, a);
+  kern<<<a.items, kSimtThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                            static_cast<const T*>(v), static_cast<const T*>(dout),
+                                            a);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
@@ -179,15 +196,20 @@ int launch_simt_backward(const void* q, const void* k, const void* v, const void
   const long long items = static_cast<long long>(s.B) * s.Hkv * a.ntk;
   if (items > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
   a.items = static_cast<int>(items);
-  const float* fq = static_cast<const float*>(q);
-  const float* fk = static_cast<const float*>(k);
-  const float* fv = static_cast<const float*>(v);
-  const float* fg = static_cast<const float*>(dout);
-  if (s.d_qk == 64 && s.d_v == 64) return launch_simt_bwd_typed<64, 64>(fq, fk, fv, fg, a, stream);
+  if (s.dtype == RA_BF16) {  // the head dims the tensor-core kernel cannot hold
+    if (s.d_qk == 192 && s.d_v == 128)
+      return launch_simt_bwd_typed<__nv_bfloat16, 192, 128>(q, k, v, dout, a, stream);
+    if (s.d_qk == 192 && s.d_v == 64)
+      return launch_simt_bwd_typed<__nv_bfloat16, 192, 64>(q, k, v, dout, a, stream);
+    return RA_ERR_UNSUPPORTED;
+  }
+  if (s.d_qk == 64 && s.d_v == 64) return launch_simt_bwd_typed<float, 64, 64>(q, k, v, dout, a, stream);
   if (s.d_qk == 128 && s.d_v == 128)
-    return launch_simt_bwd_typed<128, 128>(fq, fk, fv, fg, a, stream);
-  if (s.d_qk == 64 && s.d_v == 128) return launch_simt_bwd_typed<64, 128>(fq, fk, fv, fg, a, stream);
-  if (s.d_qk == 128 && s.d_v == 64) return launch_simt_bwd_typed<128, 64>(fq, fk, fv, fg, a, stream);
+    return launch_simt_bwd_typed<float, 128, 128>(q, k, v, dout, a, stream);
+  if (s.d_qk == 64 && s.d_v == 128)
+    return launch_simt_bwd_typed<float, 64, 128>(q, k, v, dout, a, stream);
+  if (s.d_qk == 128 && s.d_v == 64)
+    return launch_simt_bwd_typed<float, 128, 64>(q, k, v, dout, a, stream);
   return RA_ERR_UNSUPPORTED;
 }
 

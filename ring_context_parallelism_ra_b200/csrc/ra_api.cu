@@ -86,7 +86,10 @@ int check_ring_args(const void* q, const void* k, const void* v, int P, int caus
 }
 
 int check_backward_dims(const ra_shape* s) {
-  if ((s->d_qk == 64 || s->d_qk == 128) && (s->d_v == 64 || s->d_v == 128)) return RA_OK;
+  // d_qk = 192 as the forward supports it: bf16 inputs only
+  if (s->d_qk == 192 && s->dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
+  if ((s->d_qk == 64 || s->d_qk == 128 || s->d_qk == 192) && (s->d_v == 64 || s->d_v == 128))
+    return RA_OK;
   return RA_ERR_UNSUPPORTED;
 }
 

@@ -141,7 +141,8 @@ def test_backward_validation_rejects_bad_arguments_before_launch():
         assert ring(fn, s, P=3) == INV                       # 128 % 3
         assert ring(fn, s, causal=2) == INV
         assert ring(fn, _shape(n_k=64)) == INV               # n_q != n_k
-        assert ring(fn, _shape(d_qk=192)) == UNS             # no backward for D_qk = 192
+        assert ring(fn, _shape(d_qk=96)) == UNS              # head dims outside {64, 128, 192}
+        assert ring(fn, _shape(dtype=ra.RA_F32, d_qk=192)) == UNS   # as the forward: bf16 only
         assert ring(fn, _shape(dtype=ra.RA_F32, d_v=32)) == UNS
         assert ring(fn, s, wsb=ctypes.c_size_t(ws - 1)) == INV
     # striped needs whole 128-row tiles per partition
@@ -158,7 +159,7 @@ def test_backward_validation_rejects_bad_arguments_before_launch():
     assert blk(s, st=0) == INV
     assert blk(s, causal=3) == INV
     assert blk(_shape(Hq=3, Hkv=2)) == INV
-    assert blk(_shape(d_qk=192)) == UNS
+    assert blk(_shape(d_qk=96)) == UNS
     assert blk(s, wsb=ctypes.c_size_t(0)) == INV
     assert L.ra_backward_delta(nul, p, ctypes.byref(s), p, nul) == INV
     assert L.ra_backward_delta(p, p, None, p, nul) == INV

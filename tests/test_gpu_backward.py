@@ -53,6 +53,8 @@ RING_CASES = [
     (1, 2, 2, 96, 128, 128, 8, True, BF),     # 12-token partitions
     (1, 2, 1, 16, 128, 128, 16, True, BF),    # one token per partition
     (1, 1, 1, 1, 128, 128, 1, True, BF),      # a single token: every gradient is 0 but dV
+    (1, 4, 2, 320, 192, 128, 2, True, BF),    # MLA-shaped head: exact-fp32 CUDA-core kernel
+    (1, 2, 2, 200, 192, 64, 4, False, BF),
 ]
 
 
@@ -86,22 +88,22 @@ def test_backward_delta_matches_oracle(dt):
     assert err.max() <= 1e-4 * max(1.0, np.abs(want).max())
 
 
-@pytest.mark.parametrize("dt", [BF, F32])
-def test_block_backward_shares_sum_to_the_gradient(dt):
+@pytest.mark.parametrize("dt,d,dvd", [(BF, 128, 128), (F32, 128, 128), (BF, 192, 128)])
+def test_block_backward_shares_sum_to_the_gradient(dt, d, dvd):
     # Device i of a P-way ring holds Q_i, dO_i and the final LSE_i, D_i; each
     # KV_j that passes adds its share to dQ_i and to the travelling dK_j, dV_j.
     # Every block is called, the fully masked ones included.
-    B, Hq, Hkv, n, d, P = 1, 4, 2, 512, 128, 4
+    B, Hq, Hkv, n, P = 1, 4, 2, 512, 4
     L = n // P
-    q, k, v = make_qkv(B, Hq, Hkv, n, n, d, d, dt, seed=11)
-    g = make_dout(B, Hq, n, d, dt, seed=11)
+    q, k, v = make_qkv(B, Hq, Hkv, n, n, d, dvd, dt, seed=11)
+    g = make_dout(B, Hq, n, dvd, dt, seed=11)
     qd, kd, vd, gd = (x.to(DEV) for x in (q, k, v, g))
     out, lse = ra.ring_forward(qd, kd, vd, P, True)
     delta = ra.backward_delta(out, gd)
     part = lambda x, i: x[:, :, i * L:(i + 1) * L].contiguous()  # noqa: E731
     dq = [torch.zeros((B, Hq, L, d), device=DEV) for _ in range(P)]
     dk = [torch.zeros((B, Hkv, L, d), device=DEV) for _ in range(P)]
-    dv = [torch.zeros((B, Hkv, L, d), device=DEV) for _ in range(P)]
+    dv = [torch.zeros((B, Hkv, L, dvd), device=DEV) for _ in range(P)]
     for i in range(P):
         for s in range(P):
             j = (i - s) % P
@@ -179,7 +181,7 @@ def test_backward_causal_dependence():
 
 
 def test_backward_rejects_what_it_does_not_support():
-    q = torch.zeros((1, 1, 256, 192), device=DEV, dtype=BF)
+    q = torch.zeros((1, 1, 256, 96), device=DEV, dtype=BF)
     v = torch.zeros((1, 1, 256, 128), device=DEV, dtype=BF)
     out = torch.zeros((1, 1, 256, 128), device=DEV, dtype=BF)
     lse = torch.zeros((1, 1, 256), device=DEV)
