@@ -646,7 +646,7 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
   a.block_mode = block_mode ? 1 : 0;
   a.ctx = dev.ctx;
 
-  if (s.dtype == RA_BF16 && s.d_qk != 192) {
+  if (s.dtype == RA_BF16) {
     a.tq = a.tk = kT;
     a.ntq = L.ntq;
     a.ntk = (s.n_k + kT - 1) / kT;
@@ -671,7 +671,7 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
     else if (s.d_qk == 64 && s.d_v == 128) rc = launch_bwd_typed<64, 128>(tq, tk, tv, tdo, a, grid, stream);
     else if (s.d_qk == 128 && s.d_v == 64) rc = launch_bwd_typed<128, 64>(tq, tk, tv, tdo, a, grid, stream);
     else return RA_ERR_UNSUPPORTED;
-  } else {  // fp32, and bf16 with d_qk = 192 (its dK does not fit tensor memory)
+  } else {
     rc = launch_simt_backward(q, k, v, dout, s, a, dev, stream);
   }
   if (rc != RA_OK) return rc;

@@ -213,4 +213,46 @@ int launch_simt_backward(const void* q, const void* k, const void* v, const void
   return RA_ERR_UNSUPPORTED;
 }
 
+int launch_backward_cuda_cores(const void* q, const void* k, const void* v, const void* out,
+                               const float* lse, const void* dout, const float* delta,
+                               const ra_shape& s, int P, int q_offset, int k_offset,
+                               long long stride, int causal, int striped, float scale, void* dq,
+                               void* dk, void* dv, bool block_mode, void* workspace,
+                               const DeviceInfo& dev, cudaStream_t stream) {
+  const BwdLayout L = bwd_layout(s.B, s.Hq, s.n_q, s.d_qk);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* ws_dq = reinterpret_cast<float*>(ws + L.dq_off);
+  float* ws_nl2 = reinterpret_cast<float*>(ws + L.nl2_off);
+  float* ws_d = reinterpret_cast<float*>(ws + L.d_off);
+  int rc = launch_backward_rows(block_mode ? nullptr : out, dout, delta, lse, s, L, ws_nl2, ws_d,
+                                ws_dq, dev, stream);
+  if (rc != RA_OK) return rc;
+  BwdArgs a{};
+  a.B = s.B;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.n_q = s.n_q;
+  a.n_k = s.n_k;
+  a.P = P;
+  a.grp = s.Hq / s.Hkv;
+  a.q_offset = q_offset;
+  a.k_offset = k_offset;
+  a.causal = causal;
+  a.striped = striped;
+  a.stride = striped ? P : stride;
+  a.scale = scale;
+  a.scale_log2 = scale * kLog2e;
+  a.ntq_ws = L.ntq;
+  a.ws_dq = ws_dq;
+  a.ws_nl2 = ws_nl2;
+  a.ws_d = ws_d;
+  a.dk = dk;
+  a.dv = dv;
+  a.block_mode = block_mode ? 1 : 0;
+  a.ctx = dev.ctx;
+  rc = launch_simt_backward(q, k, v, dout, s, a, dev, stream);
+  if (rc != RA_OK) return rc;
+  return launch_dq_finalize(ws_dq, dq, s, L, scale, block_mode, stream);
+}
+
 }  // namespace ra

@@ -65,6 +65,15 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
                     int P, int q_offset, int k_offset, long long stride, int causal, int striped,
                     float scale, void* dq, void* dk, void* dv, bool block_mode, void* workspace,
                     const DeviceInfo& dev, cudaStream_t stream);
+// The same sequence as launch_backward (row statistics, gradient shares, dQ
+// conversion) with the CUDA-core gradient kernel: bf16 inputs whose d_qk = 192
+// leaves the tensor-core kernel no tensor memory for dK.
+int launch_backward_cuda_cores(const void* q, const void* k, const void* v, const void* out,
+                               const float* lse, const void* dout, const float* delta,
+                               const ra_shape& s, int P, int q_offset, int k_offset,
+                               long long stride, int causal, int striped, float scale, void* dq,
+                               void* dk, void* dv, bool block_mode, void* workspace,
+                               const DeviceInfo& dev, cudaStream_t stream);
 int launch_backward_delta(const void* out, const void* dout, const ra_shape& s, float* delta,
                           const DeviceInfo& dev, cudaStream_t stream);
 struct BwdArgs;
