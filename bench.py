@@ -24,7 +24,6 @@ import dataclasses
 import hashlib
 import re
 import json
-import math
 import os
 import statistics
 import sys

@@ -3,8 +3,6 @@ times.  The oracle checks sampled outputs one by one (rows are independent,
 so each sampled row is an exact check); every other output is checked for
 finiteness.  Inputs are drawn on the GPU (see workloads.py) and the oracle
 receives CPU copies of the slices it needs."""
-import math
-
 import numpy as np
 import pytest
 import torch
@@ -93,7 +91,7 @@ def test_backward_causal_gqa_128k_full_size():
     # sum_u dK_u = 0 and sum_u dV_u = sum_t dO_t (per column).
     from oracle.backward import attention_backward_sampled
     from ring_context_parallelism_ra_b200.workloads import make_dout
-    from tests.parity_util import check_grad, to64
+    from tests.parity_util import check_grad
     wl = workload("causal_gqa_128k")
     torch.cuda.empty_cache()
     q, k, v = make_workload_inputs(wl, device="cuda")

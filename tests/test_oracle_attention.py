@@ -5,7 +5,6 @@ with pure-Python loops, closed forms, and exact invariants of softmax
 attention.
 """
 import math
-import random
 
 import numpy as np
 import pytest
