@@ -10,7 +10,7 @@ sample, and the pass-Q decode leg (GB/s of KV cache read) that the metric
 also names.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload causal_mha_8k|causal_gqa_128k|causal_mla_256k|noncausal_fp32_512]
+                    [--workload causal_mla_256k|causal_gqa_128k|causal_mha_8k|noncausal_fp32_512]
     python bench.py --impl reference ...   # the fp64 CPU oracle, same line
 
 N > 1 (torchrun): every rank runs an independent replica of the workload
@@ -196,7 +196,7 @@ def oracle_sample(wl, budget_s, seed=0):
     dt = time.perf_counter() - t0
     desc = (f"{done_rows} random query rows of one head at n={n} (full key range each, "
             f"causal FLOPs counted per row), {dt:.1f} s")
-    return flops / dt / 1e12, cores, desc
+    return flops / dt / 1e12, cores, desc, dt
 
 
 # ------------------------------------------------------------- our arm ----
@@ -301,27 +301,21 @@ def run_ours(args, world, rank):
     others = (None if args.skip_workloads
               else run_workloads_leg(args, world, rank, args.workload, peaks, peaks_kind))
     backward = None
-    if not args.skip_backward and wl.dtype == "bf16":
-        backward = [run_backward_leg(args, world, rank, w, peaks, peaks_kind)
-                    for w in (wl, workload("causal_gqa_128k"))]
+    if not args.skip_backward:
+        backward = [run_backward_leg(args, world, rank, workload(key), peaks, peaks_kind)
+                    for key in BACKWARD_WORKLOADS]
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "seq_len": wl.n,
-                   "d_qk": wl.d_qk, "d_v": wl.d_v, "P": wl.P, "causal": wl.causal,
-                   "flops_per_step": flops, "flop_convention": "2*B*Hq*n^2*(d_qk+d_v), x1/2 causal",
-                   "l2": "flushed between timed steps (256 MiB write, outside the step events)",
-                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "config": config_of(wl, world),
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
-    if decode is not None:
-        line["decode"] = decode
     if striped is not None:
         line["striped"] = striped
     if backward is not None:
@@ -330,7 +324,23 @@ def run_ours(args, world, rank):
         line["merge"] = merge
     if others is not None:
         line["workloads"] = others
+    if decode is not None:
+        # the pass-Q decode leg goes at the end of the line (main() keeps it
+        # there), its short-cache latencies just before it
+        line["decode_short_cache"] = decode.pop("short_cache")
+        line["decode"] = decode
     return line
+
+
+def config_of(wl, world):
+    """The line's `config`; both arms print the same dict for a workload."""
+    return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "seq_len": wl.n,
+            "d_qk": wl.d_qk, "d_v": wl.d_v, "P": wl.P, "causal": wl.causal,
+            "flops_per_step": prefill_flops(wl),
+            "flop_convention": "2*B*Hq*n^2*(d_qk+d_v), x1/2 causal",
+            "l2": "GPU arm: flushed between timed steps (256 MiB write, outside the step "
+                  "events); CPU oracle arm: not applicable",
+            "parallelism": f"replicas{world}" if world > 1 else "single"}
 
 
 def alu_peak_tflops(sm_mhz, num_sms):
@@ -349,7 +359,7 @@ def run_workloads_leg(args, world, rank, main_key, peaks, peaks_kind):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     res = []
-    for key in ("noncausal_fp32_512", "causal_gqa_128k", "causal_mla_256k"):
+    for key in PREFILL_WORKLOADS:
         if key == main_key:
             continue
         wl = workload(key)
@@ -513,6 +523,11 @@ def run_backward_leg(args, world, rank, wl, peaks, peaks_kind):
 
 
 TC_FILES = ["tc_attention.cu", "ptx.cuh", "block_class.cuh"]
+# every prefill workload is timed: the headline one in the main leg, the
+# others in the `workloads` leg
+PREFILL_WORKLOADS = ("causal_mla_256k", "causal_gqa_128k", "causal_mha_8k", "noncausal_fp32_512")
+# workloads whose backward runs on the tensor-core kernel
+BACKWARD_WORKLOADS = ("causal_mha_8k", "causal_gqa_128k")
 BWD_FILES = ["bwd_attention.cu", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
 
 
@@ -695,23 +710,25 @@ def run_decode_leg(args, world, rank, peaks, peaks_kind):
 def run_reference(args, world, rank):
     wl = workload(args.workload)
     budget = float(os.environ.get("RA_ORACLE_BUDGET_S", "12"))
-    vals = []
+    vals, walls = [], []
     desc, cores = "", 0
     for i in range(args.warmup + args.steps):
         per = budget / max(1, args.steps) if i >= args.warmup else min(2.0, budget / 10)
-        val, cores, desc = oracle_sample(wl, per, seed=i)
+        val, cores, desc, dt = oracle_sample(wl, per, seed=i)
         if i >= args.warmup:
             vals.append(val)
+            walls.append(dt)
     value = statistics.mean(vals)
     flops = prefill_flops(wl)
-    ms = flops / (value * 1e12) * 1e3
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        # each step is a bounded sample of the workload: its measured wall time
+        "ms_per_step": round(statistics.mean(walls) * 1e3, 3),
+        "ms_per_step_full_workload_extrapolated": round(flops / (value * 1e12) * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "seq_len": wl.n,
-                   "d_qk": wl.d_qk, "d_v": wl.d_v, "P": wl.P, "causal": wl.causal},
+        "config": config_of(wl, world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                          "kind": "oracle", "sample": desc + " per step"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -725,7 +742,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="causal_mha_8k",
+    ap.add_argument("--workload", default="causal_mla_256k",
                     choices=["causal_mha_8k", "causal_gqa_128k", "causal_mla_256k",
                              "noncausal_fp32_512"])
     ap.add_argument("--skip-decode", action="store_true")
@@ -746,9 +763,12 @@ def main():
     world, rank, _ = dist_setup(args.gpus)
     line = run_ours(args, world, rank)
     if rank == 0:
-        val, cores, desc = oracle_sample(workload(args.workload), args.cpu_budget_s)
+        val, cores, desc, _ = oracle_sample(workload(args.workload), args.cpu_budget_s)
         line["cpu_baseline"] = {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores,
                                 "kind": "oracle", "sample": desc}
+        for key in ("decode_short_cache", "decode"):   # keep the decode leg last
+            if key in line:
+                line[key] = line.pop(key)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -7,7 +7,7 @@ and that these reproduce the pages' worked numbers.
 from __future__ import annotations
 
 __all__ = ["kv_cache_bytes", "decode_latency_lower_bound_s", "prefill_flops",
-           "backward_flops", "pass_kv_bytes_per_chip", "kv_bytes_per_chip", "mla_ckv_bytes",
+           "backward_flops", "pass_kv_bytes_per_chip", "mla_ckv_bytes",
            "prefill_compute_time_s", "prefill_time_s", "scaling_efficiency"]
 
 
@@ -46,11 +46,6 @@ def pass_kv_bytes_per_chip(cp, S, c_kv):
     """Same page, prefill section: KV bytes each chip forwards round the ring,
     (cp - 1) / cp * S * c_kv."""
     return (cp - 1) * S * c_kv / cp
-
-
-def kv_bytes_per_chip(S, cp, c_kv, L):
-    """Same page, Eq. (cpeval-capacity): S / cp * c_kv * L."""
-    return S / cp * c_kv * L
 
 
 def mla_ckv_bytes(kv_lora_rank, rope_dim, bytes_per_value):

@@ -1,6 +1,6 @@
 """Small, fixed launches of each kernel for profiler captures.
 
-    python -m ring_context_parallelism_ra_b200.profile_cases CASE [--reps N]
+    python profile_cases.py CASE [--reps N]
 
 Each case runs two warm-up launches and then N (default 1) launches of one
 kernel at a shape the bench uses, holding at most a few GB on the device
@@ -10,6 +10,9 @@ kernel's device time printed; no replay, unlike ncu):
   prefill_mha8k   fused ring forward, causal MHA, 8 heads, n = 8192, d = 128,
                  P = 4 (the bench's default workload, one launch per step)
   prefill_gqa32k fused ring forward, causal GQA 32/8 heads, n = 32768, P = 8
+  prefill_mla32k fused ring forward, causal MLA-shaped head (d_qk = 192,
+                 d_v = 128), 16 heads, n = 32768, P = 16 (the 256K workload's
+                 head shape and partition count at an eighth of its length)
   decode_shard   pass-Q decode partial on one 131072-token shard of the
                  1M-token cache (B = 4, 64/8 heads): one chunk-kernel launch
                  and one merge launch, as one shard of the bench's decode step
@@ -26,8 +29,14 @@ import argparse
 
 import torch
 
-from . import ra
-from .workloads import make_dout, make_qkv, make_workload_inputs, workload
+import os
+import sys
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+from ring_context_parallelism_ra_b200 import ra  # noqa: E402
+from ring_context_parallelism_ra_b200.workloads import (make_dout, make_qkv,  # noqa: E402
+                                                        make_workload_inputs, workload)
 
 
 # With --activity every launch starts from a cold L2, as in the bench: a
@@ -64,7 +73,8 @@ def _backward(q, k, v, P, reps):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["prefill_mha8k", "prefill_gqa32k", "decode_shard", "merge_p8",
+    ap.add_argument("case", choices=["prefill_mha8k", "prefill_gqa32k", "prefill_mla32k",
+                                     "decode_shard", "merge_p8",
                                      "merge_p4_8k", "backward_mha8k", "backward_gqa32k"])
     ap.add_argument("--reps", type=int, default=1)
     ap.add_argument("--activity", action="store_true",
@@ -93,6 +103,9 @@ def run_case(args):
     elif args.case == "prefill_gqa32k":
         q, k, v = make_qkv(1, 32, 8, 32768, 32768, 128, 128, torch.bfloat16, seed=3, device=dev)
         _prefill(q, k, v, 8, args.reps)
+    elif args.case == "prefill_mla32k":
+        q, k, v = make_qkv(1, 16, 16, 32768, 32768, 192, 128, torch.bfloat16, seed=5, device=dev)
+        _prefill(q, k, v, 16, args.reps)
     elif args.case == "backward_mha8k":
         wl = workload("causal_mha_8k")
         q, k, v = make_workload_inputs(wl, device=dev)
