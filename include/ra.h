@@ -216,7 +216,12 @@ int ra_decode_partials(const void* q, const void* k, const void* v, int P, const
  * loop that must not call cudaMalloc (which may synchronise the device).
  * The chunk partials live in one file-scope device array of 16 MiB, held on
  * every GPU that loads the library until the process exits.  The call itself
- * allocates nothing and calls no allocating routine.
+ * allocates nothing and calls no allocating routine.  The CUDA runtime
+ * commits the array's device memory when it loads the library's module on a
+ * device: at library load under eager module loading, or under lazy loading
+ * (the CUDA 12 default) at the first decode call on that device.  That first
+ * call can therefore fail with RA_ERR_CUDA when the device is out of memory;
+ * make one warm-up call at initialisation, outside any stream capture.
  *   Arguments, layout and results as ra_decode_partial, minus the workspace.
  *   Limit: ceil(n_k / 2048) * B * Hq * (d_v + 1) * 4 + 256 bytes must not
  *   exceed 16 MiB (e.g. a 131072-token shard with B * Hq = 256 needs 8.5 MB);
@@ -225,7 +230,9 @@ int ra_decode_partials(const void* q, const void* k, const void* v, int P, const
  *   that device current) and caches it; make that first call before any
  *   stream capture.  All calls share the array and it keeps the last call's
  *   contents; calls whose kernels overlap on the GPU (e.g. on two unordered
- *   streams) race on it, so order them on one stream.
+ *   streams) race on it, so order them on one stream.  The cached address
+ *   belongs to the device's primary context: do not call the library again
+ *   after cudaDeviceReset (or after the primary context was destroyed).
  * Errors: as ra_decode_partial.
  */
 int ra_decode_partial_noalloc(const void* q, const void* k_shard, const void* v_shard,
