@@ -15,6 +15,13 @@ mean-abs err <= 2e-3 * max(1, mean |ref|); fp32: 1e-4 * max(1, max |ref|).
 import numpy as np
 import torch
 
+# The tensor cores' fp32 accumulation rounds each step toward zero
+# (tests/test_gpu_accumulation.py measures it), so an accumulator that takes
+# `steps` K = 16 steps shrinks by up to about steps x 2^-24 of its size: a
+# long positive sum loses on average half an ulp per step, and an ulp is at
+# most 2^-23 of the running sum.
+ACCUM_SHRINK_PER_STEP = 2.0 ** -24
+
 BF16_MAX_ABS = 2e-2
 BF16_MEAN_ABS = 2e-3
 F32_MAX_ABS = 1e-4
@@ -71,3 +78,15 @@ def check_grad(got, want, dtype, what="grad"):
         assert mean <= BF16_MEAN_ABS * s_mean, \
             f"{what}: mean abs {mean:.3g} > {BF16_MEAN_ABS} x {s_mean:.3g}"
     return mx, mean
+
+
+def sum_identity_bar(x, steps, axis):
+    """Bar on |sum of n entries - its exact value| for entries each computed by
+    the bf16 kernels: the systematic shrinkage of the tensor cores'
+    round-toward-zero accumulation (``steps`` K-steps of the longest
+    accumulator, ACCUM_SHRINK_PER_STEP each, relative to the entries' sizes)
+    plus random rounding, which adds up like a random walk (root sum of
+    squares at the bf16 max-abs bar)."""
+    x = to64(x)
+    return (steps * ACCUM_SHRINK_PER_STEP * np.abs(x).sum(axis=axis)
+            + BF16_MAX_ABS * np.sqrt((x ** 2).sum(axis=axis)))
