@@ -63,16 +63,23 @@ static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kRegsLaunch,
 constexpr int kSmemLimit = 232448;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+constexpr int kNT = 16;             // barriers / headers of K and V loads in flight
+
 template <int DQK, int DV>
 struct Cfg {
   static constexpr int QBOX = DQK / 64;
   static constexpr int VBOX = DV / 64;
   static constexpr int QTILE = QBOX * kBox;
-  static constexpr int SLOT = (QBOX > VBOX ? QBOX : VBOX) * kBox;
-  static constexpr int NSLOT_FIT = (kSmemLimit - 2048 - 2 * QTILE) / SLOT;
-  static constexpr int NSLOT = NSLOT_FIT > 6 ? 6 : NSLOT_FIT;
-  static constexpr int SMEM = 1024 + 2 * QTILE + NSLOT * SLOT + 1024;
-  static_assert(NSLOT >= 2, "need at least two K/V slots");
+  // K and V tiles stream through a ring of 16 KB units (one TMA box each): a
+  // K tile takes QBOX units (it may wrap around the ring), a V tile VBOX
+  // units (kept contiguous: its MMA reads both boxes through one descriptor)
+  static constexpr int NUNIT_FIT = (kSmemLimit - 2048 - 2 * QTILE) / kBox;
+  static constexpr int NUNIT = NUNIT_FIT > 12 ? 12 : NUNIT_FIT;
+  static constexpr int SMEM = 1024 + 2 * QTILE + NUNIT * kBox + 1024;
+  // V(j) and K(j+1) are in use together; a V tile may skip up to VBOX - 1
+  // units at the end of the ring
+  static_assert(NUNIT >= QBOX + 2 * VBOX - 1, "K/V ring too small");
+  static_assert(NUNIT <= kNT, "every unit's last load must keep its barrier");
   static_assert(SMEM <= kSmemLimit, "shared memory budget");
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, kBN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, DV, 0, 1);
@@ -192,14 +199,40 @@ struct TileWalk {
 // Descriptors of successive K steps differ only in the start-address field
 // (bits 0-13, address >> 4), which never carries out for shared memory, so
 // they are formed by adding (byte offset >> 4) to the tile's base descriptor.
+// First unit of the next K (contiguous = false) or V (contiguous = true) tile
+// of `n` units; producer and MMA thread run the same sequence of calls.
+template <int NUNIT>
+__device__ __forceinline__ int alloc_units(int& pos, int n, bool contiguous) {
+  if (contiguous && pos + n > NUNIT) pos = 0;
+  const int u0 = pos;
+  pos += n;
+  if (pos >= NUNIT) pos -= NUNIT;
+  return u0;
+}
+
+// Header of a K load, written by the producer before the load is armed:
+// the two query tiles' classes and whether it is the item's last K/V tile.
+__device__ __forceinline__ uint32_t tile_header(const int8_t (&cls)[2], bool last) {
+  return static_cast<uint32_t>(static_cast<uint8_t>(cls[0])) |
+         (static_cast<uint32_t>(static_cast<uint8_t>(cls[1])) << 8) | (last ? (1u << 16) : 0u);
+}
+
 template <int DQK, int DV>
-__device__ __forceinline__ void issue_s(uint32_t tmem_d, uint32_t q_base, uint32_t k_base) {
+__device__ __forceinline__ void issue_s(uint32_t tmem_d, uint32_t q_base, uint32_t kv_base,
+                                        int ku0) {
+  using C = Cfg<DQK, DV>;
   const uint64_t da = sdesc_k_sw128(q_base);
-  const uint64_t db = sdesc_k_sw128(k_base);
+  uint64_t db[C::QBOX];
+#pragma unroll
+  for (int b = 0; b < C::QBOX; ++b) {
+    const int u = ku0 + b < C::NUNIT ? ku0 + b : ku0 + b - C::NUNIT;
+    db[b] = sdesc_k_sw128(kv_base + u * kBox);
+  }
 #pragma unroll
   for (int ks = 0; ks < DQK / 16; ++ks) {
-    const uint32_t off = ((ks >> 2) * kBox + (ks & 3) * 32) >> 4;
-    umma_ss(tmem_d, da + off, db + off, Cfg<DQK, DV>::IDESC_S, ks > 0 ? 1u : 0u);
+    const uint32_t qoff = ((ks >> 2) * kBox + (ks & 3) * 32) >> 4;
+    const uint32_t koff = ((ks & 3) * 32) >> 4;
+    umma_ss(tmem_d, da + qoff, db[ks >> 2] + koff, C::IDESC_S, ks > 0 ? 1u : 0u);
   }
 }
 
@@ -219,18 +252,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, TcArgs a) {
   using C = Cfg<DQK, DV>;
-  constexpr int NSLOT = C::NSLOT;
+  constexpr int NUNIT = C::NUNIT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = sm;
   uint8_t* sKV = sm + 2 * C::QTILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NSLOT * C::SLOT);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NUNIT * kBox);
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
-  uint64_t* slot_full = bars + 2;
-  uint64_t* slot_empty = slot_full + NSLOT;
-  uint64_t* s_full = slot_empty + NSLOT;
+  uint64_t* ld_full = bars + 2;          // [kNT] K / V load L landed
+  uint64_t* ld_empty = ld_full + kNT;    // [kNT] load L consumed by the tensor cores
+  uint64_t* s_full = ld_empty + kNT;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* drain = o_full + 2;
@@ -238,6 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* kv_issued = abort_flag + 1;
   volatile int* q_issued = abort_flag + 2;
+  volatile uint32_t* item_has_tiles = reinterpret_cast<volatile uint32_t*>(abort_flag + 3);
+  volatile uint32_t* hdr = item_has_tiles + 1;  // [kNT] headers of K loads
+  int* unit_owner = const_cast<int*>(reinterpret_cast<volatile int*>(hdr + kNT));  // [NUNIT]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -245,10 +281,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < NSLOT; ++s) {
-      mbar_init(&slot_full[s], 1);
-      mbar_init(&slot_empty[s], 1);
+    for (int s = 0; s < kNT; ++s) {
+      mbar_init(&ld_full[s], 1);
+      mbar_init(&ld_empty[s], 1);
     }
+    for (int u = 0; u < NUNIT; ++u) unit_owner[u] = -1;
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], kBM);
@@ -271,53 +308,88 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
   if (warp >= 8) regs_dec<kRegsOther>();
   if (warp == 8) {
     // ------------------------------------------------------ TMA producer --
+    // Walks each item's tiles one ahead, so that every K load carries the
+    // header the MMA thread needs (classes, last tile of the item); a unit
+    // is refilled once the load that last used it has been consumed.
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       uint32_t ld = 0, qi = 0;
+      int pos = 0;
       Item it;
-      for (int round = 0; !*abort_flag && item_at(a, round, it); ++round) {
+      bool ok = true;
+      // claim `n` units from `u0` for load L: wait until their previous
+      // loads have been consumed
+      auto claim = [&](int u0, int n, uint32_t L) -> bool {
+        int waited = -1;
+        for (int b = 0; b < n; ++b) {
+          const int u = u0 + b < NUNIT ? u0 + b : u0 + b - NUNIT;
+          const int o = unit_owner[u];
+          if (o >= 0 && o != waited) {
+            if (!mbar_wait(&ld_empty[o % kNT], (static_cast<uint32_t>(o) / kNT) & 1, a.ctx,
+                           abort_flag))
+              return false;
+            waited = o;
+          }
+          unit_owner[u] = static_cast<int>(L);
+        }
+        return true;
+      };
+      for (int round = 0; ok && !*abort_flag && item_at(a, round, it); ++round) {
         if (!mbar_wait(q_empty, (qi & 1) ^ 1, a.ctx, abort_flag)) break;
+        TileWalk w;
+        w.start(a, it);
+        int kt, klen, nkt, nklen;
+        long long koff, nkoff;
+        int8_t cls[2], ncls[2];
+        bool have = w.next(a, it, kt, klen, koff, cls);
+        *item_has_tiles = have ? 1u : 0u;
         mbar_arrive_expect_tx(q_full, 2 * C::QTILE);
         for (int t = 0; t < 2; ++t)
           for (int bx = 0; bx < C::QBOX; ++bx)
             tma_load_3d(sQ + t * C::QTILE + bx * kBox, &tm_q, q_full, bx * 64, it.q0[t], it.bh);
         *q_issued = static_cast<int>(++qi);
         const int bkv = it.b * a.Hkv + it.g;
-        TileWalk w;
-        w.start(a, it);
-        int kt, klen;
-        long long koff;
-        int8_t cls[2];
-        bool ok = true;
-        while (ok && w.next(a, it, kt, klen, koff, cls)) {
-          for (int part = 0; part < 2 && ok; ++part) {  // K then V
-            const int s = ld % NSLOT;
-            if (!mbar_wait(&slot_empty[s], ((ld / NSLOT) & 1) ^ 1, a.ctx, abort_flag)) {
-              ok = false;
-              break;
-            }
-            uint8_t* dst = sKV + s * C::SLOT;
-            if (part == 0) {
-              mbar_arrive_expect_tx(&slot_full[s], C::QBOX * kBox);
-              for (int bx = 0; bx < C::QBOX; ++bx)
-                tma_load_3d(dst + bx * kBox, &tm_k, &slot_full[s], bx * 64, kt, bkv);
-            } else {
-              mbar_arrive_expect_tx(&slot_full[s], C::VBOX * kBox);
-              for (int bx = 0; bx < C::VBOX; ++bx)
-                tma_load_3d(dst + bx * kBox, &tm_v, &slot_full[s], bx * 64, kt, bkv);
-            }
-            *kv_issued = static_cast<int>(++ld);
+        while (have) {
+          const bool nhave = w.next(a, it, nkt, nklen, nkoff, ncls);
+          // K tile: may wrap around the ring
+          uint32_t L = ld;
+          int u0 = alloc_units<NUNIT>(pos, C::QBOX, false);
+          if (!(ok = claim(u0, C::QBOX, L))) break;
+          hdr[L % kNT] = tile_header(cls, !nhave);
+          mbar_arrive_expect_tx(&ld_full[L % kNT], C::QBOX * kBox);
+          for (int bx = 0; bx < C::QBOX; ++bx) {
+            const int u = u0 + bx < NUNIT ? u0 + bx : u0 + bx - NUNIT;
+            tma_load_3d(sKV + u * kBox, &tm_k, &ld_full[L % kNT], bx * 64, kt, bkv);
           }
+          *kv_issued = static_cast<int>(++ld);
+          // V tile: contiguous units
+          L = ld;
+          u0 = alloc_units<NUNIT>(pos, C::VBOX, true);
+          if (!(ok = claim(u0, C::VBOX, L))) break;
+          mbar_arrive_expect_tx(&ld_full[L % kNT], C::VBOX * kBox);
+          for (int bx = 0; bx < C::VBOX; ++bx)
+            tma_load_3d(sKV + (u0 + bx) * kBox, &tm_v, &ld_full[L % kNT], bx * 64, kt, bkv);
+          *kv_issued = static_cast<int>(++ld);
+          have = nhave;
+          kt = nkt;
+          klen = nklen;
+          koff = nkoff;
+          cls[0] = ncls[0];
+          cls[1] = ncls[1];
         }
-        if (!ok) break;
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------- MMA issuer --
+    // Follows the producer's loads in order (same unit allocation), reading
+    // each K load's header instead of walking the tiles itself: the issuing
+    // thread does as little as possible between batches of MMAs, since the
+    // tensor pipe idles as soon as its short instruction queue drains.
     if (lane == 0) {
       uint32_t ld = 0, qi = 0, pph[2] = {0, 0};
+      int pos = 0;
       const uint32_t q_base[2] = {smem_u32(sQ), smem_u32(sQ + C::QTILE)};
       const uint32_t kv_base = smem_u32(sKV);
       Item it;
@@ -326,66 +398,64 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
         if (!(ok = mbar_wait(q_full, qi & 1, a.ctx, abort_flag))) break;
         ++qi;
         tc_fence_after();
-        TileWalk w;
-        w.start(a, it);
-        int kt, klen;
-        long long koff;
-        int8_t cls[2], ncls[2];
         bool any[2] = {false, false};
-        if (w.next(a, it, kt, klen, koff, cls)) {
-          uint32_t kslot = ld % NSLOT, kph = (ld / NSLOT) & 1;
-          uint32_t vslot = (ld + 1) % NSLOT, vph = ((ld + 1) / NSLOT) & 1;
-          ld += 2;
-          if (!(ok = mbar_wait(&slot_full[kslot], kph, a.ctx, abort_flag))) break;
+        if (*item_has_tiles) {
+          uint32_t kL = ld++;
+          int ku0 = alloc_units<NUNIT>(pos, C::QBOX, false);
+          if (!(ok = mbar_wait(&ld_full[kL % kNT], (kL / kNT) & 1, a.ctx, abort_flag))) break;
           tc_fence_after();
+          uint32_t h = hdr[kL % kNT];
+          int8_t cls[2] = {static_cast<int8_t>(h & 0xff), static_cast<int8_t>((h >> 8) & 0xff)};
+          bool last = (h >> 16) & 1;
           for (int t = 0; t < 2; ++t) {
             if (cls[t] == kSkip) continue;
-            issue_s<DQK, DV>(tmem + t * 128, q_base[t], kv_base + kslot * C::SLOT);
+            issue_s<DQK, DV>(tmem + t * 128, q_base[t], kv_base, ku0);
             umma_commit(&s_full[t]);
           }
-          umma_commit(&slot_empty[kslot]);
+          umma_commit(&ld_empty[kL % kNT]);
           while (true) {
-            int nkt, nklen;
-            long long nkoff;
-            const bool has_next = w.next(a, it, nkt, nklen, nkoff, ncls);
-            uint32_t nkslot = 0, nkph = 0, nvslot = 0, nvph = 0;
-            if (has_next) {
-              nkslot = ld % NSLOT;
-              nkph = (ld / NSLOT) & 1;
-              nvslot = (ld + 1) % NSLOT;
-              nvph = ((ld + 1) / NSLOT) & 1;
-              ld += 2;
-            }
-            if (!(ok = mbar_wait(&slot_full[vslot], vph, a.ctx, abort_flag))) break;
+            const uint32_t vL = ld++;
+            const int vu0 = alloc_units<NUNIT>(pos, C::VBOX, true);
+            if (!(ok = mbar_wait(&ld_full[vL % kNT], (vL / kNT) & 1, a.ctx, abort_flag))) break;
             tc_fence_after();
             bool k_ready = false;
+            int8_t ncls[2] = {kSkip, kSkip};
+            bool nlast = true;
             for (int t = 0; t < 2 && ok; ++t) {
               if (cls[t] != kSkip) {
                 if (!(ok = mbar_wait(&p_full[t], pph[t] & 1, a.ctx, abort_flag))) break;
                 ++pph[t];
                 tc_fence_after();
-                issue_pv<DQK, DV>(tmem + 256 + t * 128, tmem + t * 128,
-                                  kv_base + vslot * C::SLOT, any[t]);
+                issue_pv<DQK, DV>(tmem + 256 + t * 128, tmem + t * 128, kv_base + vu0 * kBox,
+                                  any[t]);
                 any[t] = true;
               }
-              if (has_next && ncls[t] != kSkip) {
+              if (!last) {
                 if (!k_ready) {
-                  if (!(ok = mbar_wait(&slot_full[nkslot], nkph, a.ctx, abort_flag))) break;
+                  kL = ld++;
+                  ku0 = alloc_units<NUNIT>(pos, C::QBOX, false);
+                  if (!(ok = mbar_wait(&ld_full[kL % kNT], (kL / kNT) & 1, a.ctx, abort_flag)))
+                    break;
                   tc_fence_after();
+                  h = hdr[kL % kNT];
+                  ncls[0] = static_cast<int8_t>(h & 0xff);
+                  ncls[1] = static_cast<int8_t>((h >> 8) & 0xff);
+                  nlast = (h >> 16) & 1;
                   k_ready = true;
                 }
-                issue_s<DQK, DV>(tmem + t * 128, q_base[t], kv_base + nkslot * C::SLOT);
-                umma_commit(&s_full[t]);
+                if (ncls[t] != kSkip) {
+                  issue_s<DQK, DV>(tmem + t * 128, q_base[t], kv_base, ku0);
+                  umma_commit(&s_full[t]);
+                }
               }
             }
             if (!ok) break;
-            umma_commit(&slot_empty[vslot]);
-            if (!has_next) break;
-            umma_commit(&slot_empty[nkslot]);
-            kslot = nkslot; kph = nkph; vslot = nvslot; vph = nvph;
-            kt = nkt; klen = nklen; koff = nkoff;
+            umma_commit(&ld_empty[vL % kNT]);
+            if (last) break;
+            umma_commit(&ld_empty[kL % kNT]);
             cls[0] = ncls[0];
             cls[1] = ncls[1];
+            last = nlast;
           }
           if (!ok) break;
         }
@@ -566,9 +636,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
   if (*abort_flag && threadIdx.x == 0) {
     // let in-flight TMA loads land before shared memory is released (bounded)
     const int n = *kv_issued;
-    for (int i = n - NSLOT < 0 ? 0 : n - NSLOT; i < n; ++i) {
+    for (int i = n - kNT < 0 ? 0 : n - kNT; i < n; ++i) {
       const unsigned long long t0 = globaltimer_ns();
-      while (!mbar_try_wait(&slot_full[i % NSLOT], (i / NSLOT) & 1) &&
+      while (!mbar_try_wait(&ld_full[i % kNT], (i / kNT) & 1) &&
              globaltimer_ns() - t0 < a.ctx.wait_ns) {
       }
     }
