@@ -26,7 +26,8 @@
 // launch allocation would never proceed; the launcher checks the compiled
 // register count against the split before every launch.)
 // Work item = 256 query rows (two 128-row tiles) of one (batch, head); items
-// are dealt heaviest first in snake order across the persistent CTAs.
+// are dealt in blocks of KV heads whose K/V fit in L2, heaviest first within
+// a block, in snake order across the persistent CTAs.
 //
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [  0,128) S0 = Q0 K^T   (P0 as packed bf16 over its first 64 columns)
@@ -94,6 +95,8 @@ struct TcArgs {
   void* out;          // [B*Hq, n_q, DV] bf16 or fp32
   float* lse;         // [B*Hq, n_q] or null
   int n_pairs, items;
+  int Lq, Lk;         // rows / keys per partition (n_q / P, n_k / P)
+  int kv_block;       // (batch, KV head)s per block of items (see item_at)
   DevCtx ctx;
 };
 
@@ -110,19 +113,31 @@ struct Item {
 // index inside the partition) is token (R - p * L) * P + p = R * P + p * (1 -
 // L * P).
 __device__ __forceinline__ long long pos_stride(const TcArgs& a) { return a.stride; }
-__device__ __forceinline__ long long part_offset(const TcArgs& a, int p, int n, int base) {
-  return a.striped ? static_cast<long long>(p) * (1 - static_cast<long long>(n / a.P) * a.P)
+__device__ __forceinline__ long long part_offset(const TcArgs& a, int p, int len, int base) {
+  return a.striped ? static_cast<long long>(p) * (1 - static_cast<long long>(len) * a.P)
                    : static_cast<long long>(base);
 }
 
 __device__ __forceinline__ bool item_at(const TcArgs& a, int round, Item& it) {
-  const int G = gridDim.x;
+  const int nc = gridDim.x;
   const int c = blockIdx.x;
-  const long long idx = static_cast<long long>(round) * G + ((round & 1) ? (G - 1 - c) : c);
+  const long long idx = static_cast<long long>(round) * nc + ((round & 1) ? (nc - 1 - c) : c);
   if (idx >= a.items) return false;
-  const int bhs = a.B * a.Hq;
-  const int r = static_cast<int>(idx / bhs);
-  it.bh = static_cast<int>(idx % bhs);
+  // Items are dealt in blocks of kv_block (batch, KV head)s whose K and V
+  // fit in L2 together: every item of a block -- heaviest pairs first, the
+  // query heads of the block next to each other -- before the next block's,
+  // so the CTAs that run at the same time stream the same K/V tiles.
+  const int G = a.Hq / a.Hkv;
+  const int n_kv = a.B * a.Hkv;
+  const long long per_kv = static_cast<long long>(a.n_pairs) * G;
+  const int blk = static_cast<int>(idx / (per_kv * a.kv_block));
+  const int kv0 = blk * a.kv_block;
+  const int hb = n_kv - kv0 < a.kv_block ? n_kv - kv0 : a.kv_block;
+  const long long in_blk = idx - static_cast<long long>(kv0) * per_kv;
+  const int r = static_cast<int>(in_blk / (static_cast<long long>(G) * hb));
+  const int within = static_cast<int>(in_blk % (static_cast<long long>(G) * hb));
+  const int kvh = kv0 + within / G;
+  it.bh = (kvh / a.Hkv) * a.Hq + (kvh % a.Hkv) * G + within % G;
   // heaviest pairs first when causal: work grows with the row's token
   // position, i.e. with the pair index (contiguous) or with the pair index
   // inside its partition (striped, all partitions' pairs of one index together)
@@ -142,10 +157,9 @@ __device__ __forceinline__ bool item_at(const TcArgs& a, int round, Item& it) {
     const int rem = a.n_q - it.q0[t];
     it.qlen[t] = rem <= 0 ? 0 : (rem < kBM ? rem : kBM);
   }
-  const int Lq = a.n_q / a.P;
-  const int i = it.q0[0] / Lq;
+  const int i = it.q0[0] / a.Lq;
   it.i = i < a.P - 1 ? i : a.P - 1;
-  it.qoff = part_offset(a, it.i, a.n_q, a.q_offset);
+  it.qoff = part_offset(a, it.i, a.Lq, a.q_offset);
   return true;
 }
 
@@ -154,26 +168,24 @@ struct TileWalk {
   int s, j, kt, kend;
   long long koff;  // key position = koff + key index * stride, partition j
   __device__ __forceinline__ void start(const TcArgs& a, const Item& it) {
-    const int Lk = a.n_k / a.P;
     s = 0;
     j = it.i;
-    kt = j * Lk;
-    kend = kt + Lk;
-    koff = part_offset(a, j, a.n_k, a.k_offset);
+    kt = j * a.Lk;
+    kend = kt + a.Lk;
+    koff = part_offset(a, j, a.Lk, a.k_offset);
   }
   // Next tile with at least one active query tile: kt0, klen, the partition's
   // key offset and the class per query tile.
   __device__ __forceinline__ bool next(const TcArgs& a, const Item& it, int& kt0, int& klen,
                                        long long& koff_out, int8_t (&cls)[2]) {
-    const int Lk = a.n_k / a.P;
     const long long st = pos_stride(a);
     while (true) {
       if (kt >= kend) {
         if (++s >= a.P) return false;
-        j = (it.i - s + a.P) % a.P;
-        kt = j * Lk;
-        kend = kt + Lk;
-        koff = part_offset(a, j, a.n_k, a.k_offset);
+        j = j == 0 ? a.P - 1 : j - 1;
+        kt = j * a.Lk;
+        kend = kt + a.Lk;
+        koff = part_offset(a, j, a.Lk, a.k_offset);
         continue;
       }
       const int len = kend - kt < kBN ? kend - kt : kBN;
@@ -184,6 +196,53 @@ struct TileWalk {
       if (cls[0] == kSkip && cls[1] == kSkip) {
         // key positions only grow inside a partition: with a causal mask
         // nothing later in this partition is visible either
+        if (a.causal) kt = kend; else kt += kBN;
+        continue;
+      }
+      kt0 = kt;
+      klen = len;
+      koff_out = koff;
+      kt += kBN;
+      return true;
+    }
+  }
+};
+
+// The tiles one query tile visits, in the same ring order as TileWalk but
+// only those whose class for this query tile is not SKIP (exactly the tiles
+// whose S the MMA thread computes for it).  Used by the softmax warpgroups;
+// scalar state only, so nothing of it lands in local memory.
+struct RowWalk {
+  int s, j, kt, kend, i;
+  long long koff, q0, qlen, qoff;
+  __device__ __forceinline__ void start(const TcArgs& a, const Item& it, int t) {
+    q0 = t ? it.q0[1] : it.q0[0];
+    qlen = t ? it.qlen[1] : it.qlen[0];
+    qoff = it.qoff;
+    i = it.i;
+    s = 0;
+    j = i;
+    kt = j * a.Lk;
+    kend = qlen > 0 ? kt + a.Lk : kt;   // a tile without rows visits nothing
+    if (qlen <= 0) s = a.P;
+    koff = part_offset(a, j, a.Lk, a.k_offset);
+  }
+  __device__ __forceinline__ bool next(const TcArgs& a, int& kt0, int& klen, long long& koff_out,
+                                       int8_t& cls) {
+    const long long st = pos_stride(a);
+    while (true) {
+      if (kt >= kend) {
+        if (++s >= a.P) return false;
+        j = j == 0 ? a.P - 1 : j - 1;
+        kt = j * a.Lk;
+        kend = kt + a.Lk;
+        koff = part_offset(a, j, a.Lk, a.k_offset);
+        continue;
+      }
+      const int len = kend - kt < kBN ? kend - kt : kBN;
+      cls = tile_class(q0, qlen, kt, len, qoff, koff, a.causal, st);
+      if (cls == kSkip) {
+        // key positions only grow inside a partition
         if (a.causal) kt = kend; else kt += kBN;
         continue;
       }
@@ -484,13 +543,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
       float m = -INFINITY, l = 0.f;
       bool any = false;
       const long long st = pos_stride(a);
-      TileWalk w;
-      w.start(a, it);
+      RowWalk w;
+      w.start(a, it, t);
       int kt, klen;
       long long koff;
-      int8_t cls[2];
-      while (w.next(a, it, kt, klen, koff, cls)) {
-        if (cls[t] == kSkip) continue;
+      int8_t cls;
+      while (w.next(a, kt, klen, koff, cls)) {
         if (!(ok = mbar_wait(&s_full[t], sph & 1, a.ctx, abort_flag))) break;
         ++sph;
         tc_fence_after();
@@ -504,10 +562,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
         reg_fence32(s + 32);
         reg_fence32(s + 64);
         reg_fence32(s + 96);
-        if (cls[t] == kPartial || klen < kBN) {
+        if (cls == kPartial || klen < kBN) {
           long long lim = klen;
           if (a.causal) {
-            const long long vis = visible_keys(it.q0[t] + row, kt, it.qoff, koff, st);
+            const long long vis = visible_keys(w.q0 + row, kt, w.qoff, koff, st);
             lim = vis < lim ? vis : lim;
           }
 #pragma unroll
@@ -581,8 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
       }
       if (!ok) break;
       // ---- epilogue: O / l and LSE for the rows that exist ----
-      const bool valid = row < it.qlen[t];
-      const long long orow = static_cast<long long>(it.bh) * a.n_q + it.q0[t] + row;
+      const bool valid = row < w.qlen;
+      const long long orow = static_cast<long long>(it.bh) * a.n_q + w.q0 + row;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       if (any) {
         if (!(ok = mbar_wait(&o_full[t], oph & 1, a.ctx, abort_flag))) break;
@@ -711,9 +769,17 @@ int launch_tc_attention(const void* q, const void* k, const void* v, const ra_sh
   a.out = out;
   a.lse = lse;
   a.n_pairs = (s.n_q + 2 * kBM - 1) / (2 * kBM);
+  a.Lq = s.n_q / P;
+  a.Lk = s.n_k / P;
   const long long items = static_cast<long long>(a.n_pairs) * s.B * s.Hq;
   if (items > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
   a.items = static_cast<int>(items);
+  // as many (batch, KV head)s per block of items as fit 48 MB of K and V
+  // (well inside the 126 MB L2, which the query tiles stream through too)
+  const long long kv_bytes = static_cast<long long>(s.n_k) * (s.d_qk + s.d_v) * 2;
+  const long long fit = (48ll << 20) / (kv_bytes > 0 ? kv_bytes : 1);
+  const long long n_kv = static_cast<long long>(s.B) * s.Hkv;
+  a.kv_block = static_cast<int>(fit < 1 ? 1 : (fit > n_kv ? n_kv : fit));
   a.ctx = dev.ctx;
   const int grid = a.items < dev.num_sms ? a.items : dev.num_sms;
   return out_f32 ? dispatch<true>(s.d_qk, s.d_v, tq, tk, tv, a, grid, stream)
