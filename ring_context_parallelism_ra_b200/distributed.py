@@ -8,15 +8,20 @@ has met every KV partition (page "AI æŽ¨ç†ç³»åˆ—ï¼ˆåä¸€ï¼‰ï¼šRing Attention å
 å¤šå¼  GPU å…±åŒè®¡ç®—ä¸€æ¡è¶…é•¿åºåˆ—", section "KV åœ¨ Ring ä¸­å¦‚ä½•æµåŠ¨"); the exchange of
 step s + 1 overlaps the block computation of step s (same page, section "é€šä¿¡
 å¾ˆå¤šï¼Œä¸ºä»€ä¹ˆä»ç„¶å¯èƒ½åˆ’ç®—"; page "LLMé•¿æ–‡æœ¬æŽ¨ç†Ring AttentionçŽ¯å½¢æ³¨æ„åŠ›æœºåˆ¶å®žçŽ°ä¸Ž
-ä¼˜åŒ–", section "Ring Attentionå®žçŽ°ä»£ç ä¸Žé€šä¿¡é‡å ").  The block partials are
-merged with the log-sum-exp rule at the end.  With a causal mask a contiguous
+ä¼˜åŒ–", section "Ring Attentionå®žçŽ°ä»£ç ä¸Žé€šä¿¡é‡å ").  Each block partial is folded
+into a running (O, LSE) with the log-sum-exp rule as soon as it is computed
+(the latter page's per-step update), so a rank holds two partials, not P.  With a causal mask a contiguous
 split skips the blocks wholly in the future (and leaves the devices unevenly
 loaded); the striped split of the latter page's tuning section gives rank r
 the tokens r, r + P, r + 2P, ... so that every block is about half visible.
 
 Backward: KV_j travels together with its gradient accumulators dK_j, dV_j,
 which collect one share per query partition; dQ_i collects at its rank; a
-last hop returns every accumulator to its owner.
+last hop returns every accumulator to its owner.  A rank computes its share
+of step s into a local buffer while the accumulator it must add it to is
+still on its way from the previous rank, then adds the two and sends the sum
+on: the accumulator hop overlaps the block computation instead of
+following it.
 
 Layout on every rank: q [B, Hq, L, d_qk], k [B, Hkv, L, d_qk], v [B, Hkv, L,
 d_v] with L = n / P tokens of its partition, in position order.  Rank r is
@@ -68,8 +73,8 @@ class KernelBlocks:
     def partial(self, q, k, v, q_offset, k_offset, stride, causal, scale, o, lse):
         return ra.block_partial_strided(q, k, v, q_offset, k_offset, stride, causal, scale, o, lse)
 
-    def merge(self, o_parts, lse_parts, out_dtype):
-        return ra.lse_merge(o_parts, lse_parts, out_dtype)
+    def merge(self, o_parts, lse_parts, out_dtype, out=None, lse=None):
+        return ra.lse_merge(o_parts, lse_parts, out_dtype, out, lse)
 
     def delta(self, out, dout):
         return ra.backward_delta(out, dout)
@@ -231,24 +236,38 @@ def ring_attention_forward(q, k, v, causal=True, scale=None, striped=False, grou
     B, Hq, L, _ = q.shape
     dv = v.shape[-1]
     scale = q.shape[-1] ** -0.5 if scale is None else scale
-    o_parts = torch.empty((P, B, Hq, L, dv), device=q.device, dtype=torch.float32)
-    l_parts = torch.empty((P, B, Hq, L), device=q.device, dtype=torch.float32)
+    # the steps whose block is computed (a contiguous causal split skips the
+    # blocks wholly in the future)
+    todo = [s for s in range(P) if not (causal and not striped and (i - s) % P > i)]
+    # running (O, LSE): slot 0 of a stack holds it, slot 1 the new block
+    # partial; the merge writes the next running value into the other stack
+    o_st = [torch.empty((2, B, Hq, L, dv), device=q.device, dtype=torch.float32)
+            for _ in range(2 if len(todo) > 1 else 1)]
+    l_st = [torch.empty((2, B, Hq, L), device=q.device, dtype=torch.float32) for _ in o_st]
     cur = [k.contiguous(), v.contiguous()]
     nbuf = [torch.empty_like(cur[0]), torch.empty_like(cur[1])]
     q_off, stride = partition_positions(i, P, L, striped)
-    used = 0
+    run, done, result = 0, 0, None
     for s in range(P):
         j = (i - s) % P
         handle = transport.exchange(cur, nbuf, nxt, prv) if s < P - 1 else _Done()
         k_off, _ = partition_positions(j, P, L, striped)
-        if not (causal and not striped and j > i):  # wholly in the future: skipped
+        if s in todo:
+            slot = 0 if done == 0 else 1
             blocks.partial(q, cur[0], cur[1], q_off, k_off, stride, causal, scale,
-                           o_parts[used], l_parts[used])
-            used += 1
+                           o_st[run][slot], l_st[run][slot])
+            done += 1
+            if done == len(todo):     # the last fold writes the result itself
+                n = 1 if done == 1 else 2
+                result = blocks.merge(o_st[run][:n], l_st[run][:n], q.dtype)
+            elif done > 1:
+                blocks.merge(o_st[run], l_st[run], torch.float32, o_st[1 - run][0],
+                             l_st[1 - run][0])
+                run = 1 - run
         handle.wait()
         if s < P - 1:
             cur, nbuf = nbuf, cur
-    return blocks.merge(o_parts[:used], l_parts[:used], q.dtype)
+    return result
 
 
 def ring_attention_backward(q, k, v, out, lse, dout, causal=True, scale=None, striped=False,
@@ -267,27 +286,39 @@ def ring_attention_backward(q, k, v, out, lse, dout, causal=True, scale=None, st
     dq = torch.zeros(q.shape, device=q.device, dtype=torch.float32)
     kv = [k.contiguous(), v.contiguous()]
     kv_buf = [torch.empty_like(kv[0]), torch.empty_like(kv[1])]
-    acc = [torch.zeros(k.shape, device=q.device, dtype=torch.float32),
-           torch.zeros(v.shape, device=q.device, dtype=torch.float32)]
-    acc_buf = [torch.empty_like(acc[0]), torch.empty_like(acc[1])]
+    f32 = dict(device=q.device, dtype=torch.float32)
+    share = [torch.empty(k.shape, **f32), torch.empty(v.shape, **f32)]   # this step's share
+    acc_in = [torch.empty(k.shape, **f32), torch.empty(v.shape, **f32)]  # arriving accumulator
+    acc_out = [torch.empty(k.shape, **f32), torch.empty(v.shape, **f32)]  # sum sent on
     q_off, stride = partition_positions(i, P, L, striped)
     for s in range(P):
         j = (i - s) % P
-        # K, V of the next step travel while this step computes; the
-        # accumulators can only leave once this step has added its share
+        # K, V of the next step travel while this step computes
         handle = transport.exchange(kv, kv_buf, nxt, prv) if s < P - 1 else _Done()
+        # KV_j's accumulator arrives from the previous rank (which added its
+        # share in its step s - 1) while this rank sends the sum of its step
+        # s - 1; at s = 0 KV_j is this rank's own and starts from zero
+        acc_h = transport.exchange(acc_out, acc_in, nxt, prv) if s > 0 else _Done()
         k_off, _ = partition_positions(j, P, L, striped)
+        share[0].zero_()
+        share[1].zero_()
         if not (causal and not striped and j > i):
             blocks.backward(q, kv[0], kv[1], dout, lse, delta, q_off, k_off, stride, causal,
-                            scale, dq, acc[0], acc[1])
-        if P > 1:
-            transport.exchange(acc, acc_buf, nxt, prv).wait()
-            acc, acc_buf = acc_buf, acc
+                            scale, dq, share[0], share[1])
+        acc_h.wait()
+        if s > 0:
+            torch.add(acc_in[0], share[0], out=acc_out[0])
+            torch.add(acc_in[1], share[1], out=acc_out[1])
+        else:
+            acc_out[0].copy_(share[0])
+            acc_out[1].copy_(share[1])
         handle.wait()
         if s < P - 1:
             kv, kv_buf = kv_buf, kv
-    # after P accumulator hops every rank holds its own dK, dV
-    return dq.to(q.dtype), acc[0].to(k.dtype), acc[1].to(v.dtype)
+    if P > 1:  # a last hop returns every accumulator to its owner
+        transport.exchange(acc_out, acc_in, nxt, prv).wait()
+        acc_out = acc_in
+    return dq.to(q.dtype), acc_out[0].to(k.dtype), acc_out[1].to(v.dtype)
 
 
 def _seq_to_heads(x, P, transport):

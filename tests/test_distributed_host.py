@@ -46,11 +46,18 @@ class OracleBlocks:
         o.copy_(torch.from_numpy(oo))
         lse.copy_(torch.from_numpy(ll))
 
-    def merge(self, o_parts, lse_parts, out_dtype):
+    def merge(self, o_parts, lse_parts, out_dtype, out=None, lse=None):
         from oracle.merge import lse_merge
         assert o_parts.is_contiguous() and lse_parts.is_contiguous()
         oo, ll = lse_merge(o_parts.double().numpy(), lse_parts.double().numpy())
-        return torch.from_numpy(oo).to(out_dtype), torch.from_numpy(ll).float()
+        o, l_ = torch.from_numpy(oo).to(out_dtype), torch.from_numpy(ll).float()
+        if out is not None:
+            out.copy_(o)
+            o = out
+        if lse is not None:
+            lse.copy_(l_)
+            l_ = lse
+        return o, l_
 
     def delta(self, out, dout):
         from oracle.backward import row_delta
@@ -161,6 +168,87 @@ def test_ring_over_gloo_matches_whole_sequence(world, striped, causal):
         errs.append(errq.get())
     assert not errs, errs
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+
+
+def _order_main(rank, world, port, errq, outq):
+    """Record, on every rank, the order in which the ring backward issues its
+    exchanges and block computations, and how many partials the forward
+    keeps alive."""
+    import torch.distributed as dist
+
+    from ring_context_parallelism_ra_b200.distributed import (HostTransport,
+                                                              ring_attention_backward,
+                                                              ring_attention_forward)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        events = []
+
+        class Rec(HostTransport):
+            def exchange(self, send, recv, nxt, prv):
+                # the travelling accumulators are fp32, K and V fp64 here
+                events.append("acc" if send[0].dtype == torch.float32 else "kv")
+                return super().exchange(send, recv, nxt, prv)
+
+        class RecBlocks(OracleBlocks):
+            def backward(self, *args):
+                events.append("block")
+                return super().backward(*args)
+
+            def merge(self, o_parts, lse_parts, out_dtype, out=None, lse=None):
+                events.append(("merge", o_parts.shape[0]))
+                return super().merge(o_parts, lse_parts, out_dtype, out, lse)
+
+        L, d = 4, 3
+        rng = np.random.default_rng(7)
+        x = lambda h: torch.from_numpy(rng.standard_normal((1, h, L, d)))  # noqa: E731
+        q, k, v, g = x(2), x(1), x(1), x(2)
+        out, lse = ring_attention_forward(q, k, v, False, 0.5, transport=Rec(), blocks=RecBlocks())
+        fwd = list(events)
+        events.clear()
+        ring_attention_backward(q, k, v, out, lse, g, False, 0.5, transport=Rec(),
+                                blocks=RecBlocks())
+        outq.put((rank, fwd, list(events)))
+    except Exception:
+        errq.put((rank, traceback.format_exc()))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ring_folds_as_it_goes_and_overlaps_the_accumulator_hop(world):
+    ctx = mp.get_context("spawn")
+    errq, outq = ctx.Queue(), ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_order_main, args=(r, world, port, errq, outq))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    errs = []
+    while not errq.empty():
+        errs.append(errq.get())
+    assert not errs, errs
+    res = [outq.get(timeout=10) for _ in range(world)]
+    for rank, fwd, bwd in res:
+        # forward: every block after the first is folded into the running
+        # result at once (two partials), never all P at the end
+        assert [e for e in fwd if e != "kv"] == [("merge", 2)] * (world - 1), (rank, fwd)
+        # backward, per step s: the next K/V leave (s < P - 1), then the
+        # accumulator of step s - 1 leaves (s > 0) -- both before this
+        # step's block is computed -- and a last hop returns the owner's sums
+        want = []
+        for s in range(world):
+            if s < world - 1:
+                want.append("kv")
+            if s > 0:
+                want.append("acc")
+            want.append("block")
+        want.append("acc")
+        assert bwd == want, (rank, bwd)
 
 
 def _ulysses_main(rank, world, port, errq):
