@@ -504,7 +504,7 @@ def run_backward_leg(args, world, rank, wl, peaks, peaks_kind):
     flops = backward_flops(wl)
     achieved = flops / (ms_local * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    tr = load_traffic(f"ring_backward:{wl.name}", BWD_FILES)
+    tr = load_traffic(f"ring_backward:{wl.name}", BWD192_FILES if wl.d_qk == 192 else BWD_FILES)
     del q, k, v, g, out, lse, ws, dq, dk, dv, flush
     torch.cuda.empty_cache()
     return {"workload": wl.name, "value": round(world * flops / (ms * 1e-3) / 1e12, 3),
@@ -517,7 +517,8 @@ def run_backward_leg(args, world, rank, wl, peaks, peaks_kind):
                          "frac_of_sustained": round(
                              achieved / peaks.get("bf16_tflops_sustained", 1400.0), 4),
                          "traffic": tr["dram_bytes_per_launch"] if tr else None,
-                         "traffic_kernel": "bwd_tc_kernel (ncu capture of the same shape)",
+                         "traffic_kernel": ("bwd_tc192_kernel" if wl.d_qk == 192 else "bwd_tc_kernel")
+                                           + " (ncu capture)",
                          "kernel": "ring_backward (prep + tcgen05 kernel + dQ conversion)"},
             "clocks": clk.summary()}
 
@@ -526,9 +527,10 @@ TC_FILES = ["tc_attention.cu", "ptx.cuh", "block_class.cuh"]
 # every prefill workload is timed: the headline one in the main leg, the
 # others in the `workloads` leg
 PREFILL_WORKLOADS = ("causal_mla_256k", "causal_gqa_128k", "causal_mha_8k", "noncausal_fp32_512")
-# workloads whose backward runs on the tensor-core kernel
-BACKWARD_WORKLOADS = ("causal_mha_8k", "causal_gqa_128k")
-BWD_FILES = ["bwd_attention.cu", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
+# the backward leg (every bf16 prefill workload; all run on the tensor cores)
+BACKWARD_WORKLOADS = ("causal_mla_256k", "causal_gqa_128k", "causal_mha_8k")
+BWD_FILES = ["bwd_attention.cu", "bwd_tc.cuh", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
+BWD192_FILES = ["bwd_tc192.cu", "bwd_tc.cuh", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
 
 
 def run_striped_leg(args, world, rank, wl, peaks):

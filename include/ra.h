@@ -263,8 +263,8 @@ int ra_decode_merge(const float* o_parts, const float* lse_parts, int P, const r
  * per query partition while dQ_i collects at its partition.
  * Supported head dims: d_qk, d_v in {64, 128} (bf16 on tensor cores, fp32
  * on the CUDA cores); bf16 d_qk = 192 with d_v in {64, 128} (the MLA-shaped
- * head) on the exact-fp32 CUDA-core kernel, since its dK accumulator does not
- * fit tensor memory beside S^T, dP^T and dV: correct, not fast.
+ * head) on tensor cores as well, its products taking turns in tensor memory
+ * (the 192-column dK accumulator leaves no room to keep S^T and dP^T apart).
  */
 
 /*

@@ -13,6 +13,11 @@ kernel's device time printed; no replay, unlike ncu):
   prefill_mla32k fused ring forward, causal MLA-shaped head (d_qk = 192,
                  d_v = 128), 16 heads, n = 32768, P = 16 (the 256K workload's
                  head shape and partition count at an eighth of its length)
+  prefill_mla256k / prefill_gqa128k
+                 fused ring forward on the full 256K MLA / 128K GQA workloads
+                 (what the bench times; for single-pass counters only)
+  backward_mla256k / backward_gqa128k
+                 ring backward on the same full-size workloads
   decode_shard   pass-Q decode partial on one 131072-token shard of the
                  1M-token cache (B = 4, 64/8 heads): one chunk-kernel launch
                  and one merge launch, as one shard of the bench's decode step
@@ -74,7 +79,8 @@ def _backward(q, k, v, P, reps):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["prefill_mha8k", "prefill_gqa32k", "prefill_mla32k",
-                                     "decode_shard", "merge_p8",
+                                     "prefill_mla256k", "prefill_gqa128k", "backward_mla256k",
+                                     "backward_gqa128k", "decode_shard", "merge_p8",
                                      "merge_p4_8k", "backward_mha8k", "backward_gqa32k"])
     ap.add_argument("--reps", type=int, default=1)
     ap.add_argument("--activity", action="store_true",
@@ -106,6 +112,14 @@ def run_case(args):
     elif args.case == "prefill_mla32k":
         q, k, v = make_qkv(1, 16, 16, 32768, 32768, 192, 128, torch.bfloat16, seed=5, device=dev)
         _prefill(q, k, v, 16, args.reps)
+    elif args.case in ("prefill_mla256k", "prefill_gqa128k"):
+        wl = workload("causal_mla_256k" if args.case == "prefill_mla256k" else "causal_gqa_128k")
+        q, k, v = make_workload_inputs(wl, device=dev)
+        _prefill(q, k, v, wl.P, args.reps)
+    elif args.case in ("backward_mla256k", "backward_gqa128k"):
+        wl = workload("causal_mla_256k" if args.case == "backward_mla256k" else "causal_gqa_128k")
+        q, k, v = make_workload_inputs(wl, device=dev)
+        _backward(q, k, v, wl.P, args.reps)
     elif args.case == "backward_mha8k":
         wl = workload("causal_mha_8k")
         q, k, v = make_workload_inputs(wl, device=dev)

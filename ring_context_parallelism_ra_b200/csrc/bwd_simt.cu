@@ -1,10 +1,9 @@
 // Exact-fp32 backward pass on the FMA pipes (no tensor cores): the same
 // gradients and the same walk as the tensor-core kernel (bwd.cuh), with
-// 64-key tiles against 64-row query tiles.  It serves fp32 inputs, and bf16
-// inputs whose d_qk = 192 leaves the tensor-core kernel no room in tensor
-// memory for the dK accumulator (inputs widened to fp32 on load; dK, dV
-// stored in the input dtype, or added into the caller's fp32 accumulators
-// for a block share).
+// 64-key tiles against 64-row query tiles.  It serves fp32 inputs (dK, dV
+// stored as fp32, or added into the caller's fp32 accumulators for a block
+// share); bf16 inputs run on the tensor cores (bwd_attention.cu,
+// bwd_tc192.cu).
 //
 // One CTA (256 threads) per key tile of one (batch, KV head).  Per visit the
 // CTA stages Q_t, dO_t and the rows' -LSE log2(e), D in shared memory, forms
@@ -32,19 +31,17 @@ struct SCfg {
 };
 
 __device__ __forceinline__ float widen(float x) { return x; }
-__device__ __forceinline__ float widen(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// Store of a finished dK / dV entry: the input dtype for the ring, or added
-// into the fp32 accumulator of a block share.
+// Store of a finished dK / dV entry: the output for the ring, or added into
+// the fp32 accumulator of a block share.
 template <typename T>
 __device__ __forceinline__ void put(void* base, long long i, float x, int block_mode) {
+  static_assert(sizeof(T) == 4, "fp32 inputs only");
   if (block_mode) {
     float* p = static_cast<float*>(base) + i;
     *p += x;
-  } else if constexpr (sizeof(T) == 4) {
-    static_cast<float*>(base)[i] = x;
   } else {
-    static_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(x);
+    static_cast<float*>(base)[i] = x;
   }
 }
 
@@ -196,13 +193,7 @@ int launch_simt_backward(const void* q, const void* k, const void* v, const void
   const long long items = static_cast<long long>(s.B) * s.Hkv * a.ntk;
   if (items > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
   a.items = static_cast<int>(items);
-  if (s.dtype == RA_BF16) {  // the head dims the tensor-core kernel cannot hold
-    if (s.d_qk == 192 && s.d_v == 128)
-      return launch_simt_bwd_typed<__nv_bfloat16, 192, 128>(q, k, v, dout, a, stream);
-    if (s.d_qk == 192 && s.d_v == 64)
-      return launch_simt_bwd_typed<__nv_bfloat16, 192, 64>(q, k, v, dout, a, stream);
-    return RA_ERR_UNSUPPORTED;
-  }
+  if (s.dtype != RA_F32) return RA_ERR_UNSUPPORTED;
   if (s.d_qk == 64 && s.d_v == 64) return launch_simt_bwd_typed<float, 64, 64>(q, k, v, dout, a, stream);
   if (s.d_qk == 128 && s.d_v == 128)
     return launch_simt_bwd_typed<float, 128, 128>(q, k, v, dout, a, stream);
@@ -211,48 +202,6 @@ int launch_simt_backward(const void* q, const void* k, const void* v, const void
   if (s.d_qk == 128 && s.d_v == 64)
     return launch_simt_bwd_typed<float, 128, 64>(q, k, v, dout, a, stream);
   return RA_ERR_UNSUPPORTED;
-}
-
-int launch_backward_cuda_cores(const void* q, const void* k, const void* v, const void* out,
-                               const float* lse, const void* dout, const float* delta,
-                               const ra_shape& s, int P, int q_offset, int k_offset,
-                               long long stride, int causal, int striped, float scale, void* dq,
-                               void* dk, void* dv, bool block_mode, void* workspace,
-                               const DeviceInfo& dev, cudaStream_t stream) {
-  const BwdLayout L = bwd_layout(s.B, s.Hq, s.n_q, s.d_qk);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* ws_dq = reinterpret_cast<float*>(ws + L.dq_off);
-  float* ws_nl2 = reinterpret_cast<float*>(ws + L.nl2_off);
-  float* ws_d = reinterpret_cast<float*>(ws + L.d_off);
-  int rc = launch_backward_rows(block_mode ? nullptr : out, dout, delta, lse, s, L, ws_nl2, ws_d,
-                                ws_dq, dev, stream);
-  if (rc != RA_OK) return rc;
-  BwdArgs a{};
-  a.B = s.B;
-  a.Hq = s.Hq;
-  a.Hkv = s.Hkv;
-  a.n_q = s.n_q;
-  a.n_k = s.n_k;
-  a.P = P;
-  a.grp = s.Hq / s.Hkv;
-  a.q_offset = q_offset;
-  a.k_offset = k_offset;
-  a.causal = causal;
-  a.striped = striped;
-  a.stride = striped ? P : stride;
-  a.scale = scale;
-  a.scale_log2 = scale * kLog2e;
-  a.ntq_ws = L.ntq;
-  a.ws_dq = ws_dq;
-  a.ws_nl2 = ws_nl2;
-  a.ws_d = ws_d;
-  a.dk = dk;
-  a.dv = dv;
-  a.block_mode = block_mode ? 1 : 0;
-  a.ctx = dev.ctx;
-  rc = launch_simt_backward(q, k, v, dout, s, a, dev, stream);
-  if (rc != RA_OK) return rc;
-  return launch_dq_finalize(ws_dq, dq, s, L, scale, block_mode, stream);
 }
 
 }  // namespace ra

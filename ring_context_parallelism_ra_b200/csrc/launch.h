@@ -2,6 +2,7 @@
 // argument validation.  Each returns an ra_status.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -65,15 +66,6 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
                     int P, int q_offset, int k_offset, long long stride, int causal, int striped,
                     float scale, void* dq, void* dk, void* dv, bool block_mode, void* workspace,
                     const DeviceInfo& dev, cudaStream_t stream);
-// The same sequence as launch_backward (row statistics, gradient shares, dQ
-// conversion) with the CUDA-core gradient kernel: bf16 inputs whose d_qk = 192
-// leaves the tensor-core kernel no tensor memory for dK.
-int launch_backward_cuda_cores(const void* q, const void* k, const void* v, const void* out,
-                               const float* lse, const void* dout, const float* delta,
-                               const ra_shape& s, int P, int q_offset, int k_offset,
-                               long long stride, int causal, int striped, float scale, void* dq,
-                               void* dk, void* dv, bool block_mode, void* workspace,
-                               const DeviceInfo& dev, cudaStream_t stream);
 int launch_backward_delta(const void* out, const void* dout, const ra_shape& s, float* delta,
                           const DeviceInfo& dev, cudaStream_t stream);
 struct BwdArgs;
@@ -87,6 +79,11 @@ int launch_dq_finalize(const float* ws_dq, void* dq, const ra_shape& s, const Bw
 int launch_simt_backward(const void* q, const void* k, const void* v, const void* dout,
                          const ra_shape& s, BwdArgs a, const DeviceInfo& dev,
                          cudaStream_t stream);
+// Gradient kernel of bf16 inputs with d_qk = 192 (bwd_tc192.cu); tensor maps
+// of q, k, v, dout as launch_backward builds them.
+int launch_bwd_tc192(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& tdo, const BwdArgs& args, int d_v, int grid,
+                     cudaStream_t stream);
 
 int launch_block_class(int n_q, int n_k, int q_block, int k_block, int q_offset, int k_offset,
                        int causal, int8_t* map_dev, cudaStream_t stream);

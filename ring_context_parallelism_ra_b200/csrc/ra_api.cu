@@ -85,13 +85,6 @@ int check_ring_args(const void* q, const void* k, const void* v, int P, int caus
   return check_attention_dims(shape);
 }
 
-// bf16 d_qk = 192 runs on the CUDA-core gradient kernel: the tensor-core
-// kernel has no tensor memory left for its dK accumulator.
-using BackwardLauncher = decltype(&launch_backward);
-BackwardLauncher backward_launcher(const ra_shape& s) {
-  return (s.dtype == RA_BF16 && s.d_qk == 192) ? launch_backward_cuda_cores : launch_backward;
-}
-
 int check_backward_dims(const ra_shape* s) {
   // d_qk = 192 as the forward supports it: bf16 inputs only
   if (s->d_qk == 192 && s->dtype != RA_BF16) return RA_ERR_UNSUPPORTED;
@@ -387,7 +380,7 @@ int ra_ring_backward(const void* q, const void* k, const void* v, const void* ou
   DeviceInfo dev;
   rc = device_info(&dev);
   if (rc != RA_OK) return rc;
-  return backward_launcher(*shape)(q, k, v, out, lse, dout, nullptr, *shape, P, 0, 0, 1, causal, 0, scale,
+  return launch_backward(q, k, v, out, lse, dout, nullptr, *shape, P, 0, 0, 1, causal, 0, scale,
                          dq, dk, dv, false, workspace, dev, static_cast<cudaStream_t>(stream));
 }
 
@@ -402,7 +395,7 @@ int ra_ring_backward_striped(const void* q, const void* k, const void* v, const 
   DeviceInfo dev;
   rc = device_info(&dev);
   if (rc != RA_OK) return rc;
-  return backward_launcher(*shape)(q, k, v, out, lse, dout, nullptr, *shape, P, 0, 0, P, causal, 1, scale,
+  return launch_backward(q, k, v, out, lse, dout, nullptr, *shape, P, 0, 0, P, causal, 1, scale,
                          dq, dk, dv, false, workspace, dev, static_cast<cudaStream_t>(stream));
 }
 
@@ -427,7 +420,7 @@ int ra_block_backward(const void* q, const void* k, const void* v, const void* d
   DeviceInfo dev;
   rc = device_info(&dev);
   if (rc != RA_OK) return rc;
-  return backward_launcher(*shape)(q, k, v, nullptr, lse, dout, delta, *shape, 1, q_offset, k_offset,
+  return launch_backward(q, k, v, nullptr, lse, dout, delta, *shape, 1, q_offset, k_offset,
                          pos_stride, causal, 0, scale, dq_acc, dk_acc, dv_acc, true, workspace,
                          dev, static_cast<cudaStream_t>(stream));
 }

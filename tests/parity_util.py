@@ -87,6 +87,11 @@ def sum_identity_bar(x, steps, axis):
     accumulator, ACCUM_SHRINK_PER_STEP each, relative to the entries' sizes)
     plus random rounding, which adds up like a random walk (root sum of
     squares at the bf16 max-abs bar)."""
+    if isinstance(x, torch.Tensor):   # reduce where the tensor lives, then fetch
+        x = x.double()
+        bar = (steps * ACCUM_SHRINK_PER_STEP * x.abs().sum(dim=axis)
+               + BF16_MAX_ABS * (x * x).sum(dim=axis).sqrt())
+        return to64(bar)
     x = to64(x)
     return (steps * ACCUM_SHRINK_PER_STEP * np.abs(x).sum(axis=axis)
             + BF16_MAX_ABS * np.sqrt((x ** 2).sum(axis=axis)))

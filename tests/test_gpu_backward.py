@@ -53,8 +53,12 @@ RING_CASES = [
     (1, 2, 2, 96, 128, 128, 8, True, BF),     # 12-token partitions
     (1, 2, 1, 16, 128, 128, 16, True, BF),    # one token per partition
     (1, 1, 1, 1, 128, 128, 1, True, BF),      # a single token: every gradient is 0 but dV
-    (1, 4, 2, 320, 192, 128, 2, True, BF),    # MLA-shaped head: exact-fp32 CUDA-core kernel
+    (1, 4, 2, 320, 192, 128, 2, True, BF),    # MLA-shaped head (its own tensor-core kernel)
     (1, 2, 2, 200, 192, 64, 4, False, BF),
+    (1, 8, 1, 257, 192, 128, 1, True, BF),    # d_qk 192: GQA 8:1, ragged tail
+    (2, 2, 2, 96, 192, 128, 8, True, BF),     # d_qk 192: 12-token partitions, batch 2
+    (1, 1, 1, 1, 192, 128, 1, True, BF),      # d_qk 192: a single token
+    (1, 2, 1, 640, 192, 64, 5, True, BF),     # d_qk 192, d_v 64, several key tiles
 ]
 
 
@@ -117,13 +121,14 @@ def test_block_backward_shares_sum_to_the_gradient(dt, d, dvd):
     check_grad(torch.cat(dv, 2), want[2], kind, "dV")
 
 
-def test_block_backward_strided_and_ragged():
+@pytest.mark.parametrize("d", [128, 192])
+def test_block_backward_strided_and_ragged(d):
     # One strided block (query partition 2, key partition 1 of a 4-way striped
     # split) with a ragged key count, against the oracle with explicit positions.
     dt, P = BF, 4
-    B, Hq, Hkv, nq, nk, d = 1, 2, 1, 200, 150, 128
-    q, k, v = make_qkv(B, Hq, Hkv, nq, nk, d, d, dt, seed=21)
-    g = make_dout(B, Hq, nq, d, dt, seed=21)
+    B, Hq, Hkv, nq, nk = 1, 2, 1, 200, 150
+    q, k, v = make_qkv(B, Hq, Hkv, nq, nk, d, 128, dt, seed=21)
+    g = make_dout(B, Hq, nq, 128, dt, seed=21)
     qp = 2 + P * np.arange(nq)
     kp = 1 + P * np.arange(nk)
     scale = 1 / math.sqrt(d)
@@ -138,11 +143,11 @@ def test_block_backward_strided_and_ragged():
     check_grad(dv, want[2], "bf16", "dV")
 
 
-@pytest.mark.parametrize("dt,n,P", [(BF, 1024, 4), (F32, 1024, 4)])
-def test_striped_ring_backward_matches_oracle(dt, n, P):
-    B, Hq, Hkv, d = 1, 2, 1, 128
-    q, k, v = make_qkv(B, Hq, Hkv, n, n, d, d, dt, seed=31)
-    g = make_dout(B, Hq, n, d, dt, seed=31)
+@pytest.mark.parametrize("dt,n,P,d", [(BF, 1024, 4, 128), (F32, 1024, 4, 128), (BF, 768, 3, 192)])
+def test_striped_ring_backward_matches_oracle(dt, n, P, d):
+    B, Hq, Hkv, dvd = 1, 2, 1, 128
+    q, k, v = make_qkv(B, Hq, Hkv, n, n, d, dvd, dt, seed=31)
+    g = make_dout(B, Hq, n, dvd, dt, seed=31)
     order = torch.tensor(striped_order(n, P))
     inv = torch.argsort(order)
     qs, ks, vs, gs = (x[:, :, order].contiguous().to(DEV) for x in (q, k, v, g))

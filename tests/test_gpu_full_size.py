@@ -83,16 +83,16 @@ def test_decode_pass_q_1m_full_size():
     torch.cuda.empty_cache()
 
 
-def test_backward_causal_gqa_128k_full_size():
-    # The ring backward on the causal GQA 128K workload in the bench's
-    # configuration: exact gradients on sampled query rows (dQ) and on the
-    # last 256 keys (dK, dV; a causal key u needs only rows t >= u), for the
-    # heads of two KV groups; identities over every key of every head:
-    # sum_u dK_u = 0 and sum_u dV_u = sum_t dO_t (per column).
+def _check_backward(key, row_seed):
+    """The ring backward on a full-size workload in the bench's configuration:
+    exact gradients on sampled query rows (dQ) and on the last 256 keys (dK,
+    dV; a causal key u needs only rows t >= u), for the query heads of the
+    first and the last KV head; identities over every key of every head:
+    sum_u dK_u = 0 and sum_u dV_u = sum_t dO_t (per column)."""
     from oracle.backward import attention_backward_sampled
     from ring_context_parallelism_ra_b200.workloads import make_dout
-    from tests.parity_util import check_grad
-    wl = workload("causal_gqa_128k")
+    from tests.parity_util import check_grad, sum_identity_bar
+    wl = workload(key)
     torch.cuda.empty_cache()
     q, k, v = make_workload_inputs(wl, device="cuda")
     g = make_dout(wl.B, wl.Hq, wl.n, wl.d_v, wl.torch_dtype, seed=wl.seed, device="cuda")
@@ -102,10 +102,12 @@ def test_backward_causal_gqa_128k_full_size():
     for t in (dq, dk, dv):
         assert torch.isfinite(t).all().item()
     G = wl.Hq // wl.Hkv
-    rows = sample_rows(wl.n, wl.P, n_uniform=24, seed=33)
+    rows = sample_rows(wl.n, wl.P, n_uniform=24, seed=row_seed)
     keys = np.arange(wl.n - 256, wl.n)
     for grp in (0, wl.Hkv - 1):
         heads = list(range(grp * G, (grp + 1) * G))
+        if G == 1:
+            heads = [grp]
         q_s, g_s = q[:, heads].cpu(), g[:, heads].cpu()
         k_s, v_s = k[:, grp:grp + 1].cpu(), v[:, grp:grp + 1].cpu()
         wq, wk, wv = attention_backward_sampled(q_s, k_s, v_s, g_s, wl.scale, True, rows, keys)
@@ -115,8 +117,7 @@ def test_backward_causal_gqa_128k_full_size():
         check_grad(dk[:, grp:grp + 1][:, :, ki], wk, "bf16", "dK last keys")
         check_grad(dv[:, grp:grp + 1][:, :, ki], wv, "bf16", "dV last keys")
     # the longest dK / dV accumulator (the first key tile of a KV head) takes
-    # G * n / 16 round-toward-zero steps in tensor memory (32768 here)
-    from tests.parity_util import sum_identity_bar
+    # G * n / 16 round-toward-zero steps in tensor memory
     steps = G * wl.n // 16
     dk64 = dk.double()
     dv64 = dv.double()
@@ -125,3 +126,12 @@ def test_backward_causal_gqa_128k_full_size():
     assert ((dv64.sum(dim=2) - want_sv).abs().cpu().numpy() <= sum_identity_bar(dv64, steps, 2)).all()
     del q, k, v, g, out, lse, dq, dk, dv, dk64, dv64
     torch.cuda.empty_cache()
+
+
+def test_backward_causal_gqa_128k_full_size():
+    _check_backward("causal_gqa_128k", 33)
+
+
+def test_backward_causal_mla_256k_full_size():
+    # the MLA-shaped head (d_qk 192, d_v 128) on its tensor-core kernel
+    _check_backward("causal_mla_256k", 35)
