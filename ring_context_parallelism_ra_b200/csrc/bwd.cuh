@@ -61,6 +61,7 @@ struct BwdArgs {
   int ntq, ntk;      // tiles per head (query tiles counted in tq rows)
   int ntq_ws;        // 128-row workspace tiles per head
   int items;         // B * Hkv * ntk
+  int kv_block;      // (batch, KV head)s per block of items (see bwd_item_at)
   float* ws_dq;
   const float* ws_nl2;
   const float* ws_d;
@@ -83,15 +84,24 @@ struct BItem {
 };
 
 // Items are dealt in snake order over the persistent CTAs, heaviest first for
-// a causal mask: low key positions are visible to the most queries.
+// a causal mask: low key positions are visible to the most queries.  They
+// come in blocks of kv_block (batch, KV head)s whose dQ accumulator fits in
+// L2 (all of a block's items before the next block's): the CTAs that run at
+// the same time then walk the same query tiles and add their dQ shares into
+// the same lines of L2, instead of spreading the reductions over a workspace
+// far larger than L2.
 __device__ __forceinline__ bool bwd_item_at(const BwdArgs& a, int round, BItem& it) {
-  const int G = gridDim.x;
+  const int nc = gridDim.x;
   const int c = blockIdx.x;
-  const long long idx = static_cast<long long>(round) * G + ((round & 1) ? (G - 1 - c) : c);
+  const long long idx = static_cast<long long>(round) * nc + ((round & 1) ? (nc - 1 - c) : c);
   if (idx >= a.items) return false;
   const int nbkv = a.B * a.Hkv;
-  const int r = static_cast<int>(idx / nbkv);
-  it.bkv = static_cast<int>(idx % nbkv);
+  const int blk = static_cast<int>(idx / (static_cast<long long>(a.ntk) * a.kv_block));
+  const int kv0 = blk * a.kv_block;
+  const int hb = nbkv - kv0 < a.kv_block ? nbkv - kv0 : a.kv_block;
+  const long long in_blk = idx - static_cast<long long>(kv0) * a.ntk;
+  const int r = static_cast<int>(in_blk / hb);
+  it.bkv = kv0 + static_cast<int>(in_blk % hb);
   int kt = r;
   if (a.striped) {  // same local tile of every partition together
     const int tpp = a.ntk / a.P;

@@ -541,6 +541,12 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
   a.dv = dv;
   a.block_mode = block_mode ? 1 : 0;
   a.ctx = dev.ctx;
+  // as many (batch, KV head)s per block of items as keep the dQ accumulator
+  // of their query heads within 48 MB (well inside the 126 MB L2)
+  const long long dq_bytes = static_cast<long long>(s.Hq / s.Hkv) * s.n_q * s.d_qk * 4;
+  const long long fit = (48ll << 20) / (dq_bytes > 0 ? dq_bytes : 1);
+  const long long nbkv = static_cast<long long>(s.B) * s.Hkv;
+  a.kv_block = static_cast<int>(fit < 1 ? 1 : (fit > nbkv ? nbkv : fit));
 
   if (s.dtype == RA_BF16) {
     a.tq = a.tk = kT;
