@@ -18,6 +18,8 @@ kernel's device time printed; no replay, unlike ncu):
                  (what the bench times; for single-pass counters only)
   backward_mla256k / backward_gqa128k
                  ring backward on the same full-size workloads
+  backward_mla32k ring backward, the MLA-shaped head at n = 32768 (as
+                 prefill_mla32k)
   decode_shard   pass-Q decode partial on one 131072-token shard of the
                  1M-token cache (B = 4, 64/8 heads): one chunk-kernel launch
                  and one merge launch, as one shard of the bench's decode step
@@ -80,7 +82,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["prefill_mha8k", "prefill_gqa32k", "prefill_mla32k",
                                      "prefill_mla256k", "prefill_gqa128k", "backward_mla256k",
-                                     "backward_gqa128k", "decode_shard", "merge_p8",
+                                     "backward_gqa128k", "backward_mla32k", "decode_shard",
+                                     "merge_p8",
                                      "merge_p4_8k", "backward_mha8k", "backward_gqa32k"])
     ap.add_argument("--reps", type=int, default=1)
     ap.add_argument("--activity", action="store_true",
@@ -120,6 +123,9 @@ def run_case(args):
         wl = workload("causal_mla_256k" if args.case == "backward_mla256k" else "causal_gqa_128k")
         q, k, v = make_workload_inputs(wl, device=dev)
         _backward(q, k, v, wl.P, args.reps)
+    elif args.case == "backward_mla32k":
+        q, k, v = make_qkv(1, 16, 16, 32768, 32768, 192, 128, torch.bfloat16, seed=5, device=dev)
+        _backward(q, k, v, 16, args.reps)
     elif args.case == "backward_mha8k":
         wl = workload("causal_mha_8k")
         q, k, v = make_workload_inputs(wl, device=dev)
