@@ -17,7 +17,9 @@
 //               dV has read P^T
 //   [192, 192 + d_v)              dV accumulator of the item
 //   [192 + d_v, 192 + d_v + 192)  dK accumulator of the item
-// so the next S^T waits until dQ has been read out: the products of a visit
+// so the next S^T waits until dQ columns 0-127 have been read out (columns
+// 128-191 are read at the next visit, before P^T is written over them, and
+// their reductions overlap that visit's dP^T and dV): the products of a visit
 // run one after another, S^T -> (P) -> dP^T, dV -> (dS) -> dQ, dK -> (dQ
 // read-out), with the exponentials, dS and the dQ reductions on the CUDA
 // cores in between.
@@ -32,8 +34,9 @@
 //   warp 1      tcgen05.mma issuer; owns the tensor-memory allocation
 //   warps 2-3   idle
 //   warps 4-11  two compute warpgroups, query columns 0-63 and 64-127 of
-//               S^T / dP^T (thread r = key r), dQ dims 0-95 and 96-191 (thread
-//               r = query r), dK / dV columns split the same way at the end
+//               S^T / dP^T (thread r = key r), dQ dims 0-63 + 128-159 and
+//               64-127 + 160-191 (thread r = query r), dK / dV columns split
+//               in halves at the end
 // Registers: 2 x 184 (compute) + 136 (warps 0-3) = 504 = 3 x 168 per lane.
 #include <cuda.h>
 
@@ -276,11 +279,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
     const int row = threadIdx.x & 127;  // TMEM lane: key (S^T, dP^T, dK, dV), query (dQ)
     const uint32_t lb = tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
     const int qc = half * 64;           // first query column of this warpgroup
-    const int dc = half * (kDQK / 2);   // first dQ / dK column of this warpgroup
+    const int dc = half * (kDQK / 2);   // first dK column of this warpgroup
+    // dQ columns of this warpgroup: [64 half, +64) inside [0, 128), read as
+    // soon as dQ is complete (the next S^T overwrites them), and [128 + 32
+    // half, +32) inside the P^T columns, read only at the next visit, just
+    // before this warpgroup writes its P^T there; their reductions then run
+    // while the tensor cores compute dP^T (off the visit's critical path)
+    const int dqa = half * 64;
+    const int dqb = 128 + half * 32;
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
     uint8_t* ds_row = sX + half * kBox + row * 128;  // atom `half`: queries qc .. qc+63
     const uint32_t sw = row & 7;
     uint32_t nv = 0, nacc = 0;
+    int tail_bh = -1, tail_qt = 0;  // visit whose dQ columns [dqb, dqb + 32) wait in TMEM
+    auto tail_dst = [&]() -> float* {
+      return a.ws_dq + bwd_dq_index(a, tail_bh, tail_qt * kT + row, dqb, kDQK);
+    };
     BItem it;
     bool ok = true;
     for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
@@ -320,6 +334,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
           for (int c = 0; c < 64; ++c)
             if (c < qm) p[c] = 0.f;
         }
+        // the previous visit's remaining dQ columns leave tensor memory
+        // before this warpgroup's P^T is written over them, and are added
+        // into the workspace while dP^T and dV run
+        uint32_t tail[32];
+        if (tail_bh >= 0) {
+          tmem_ld32(lb + C::DQ + dqb, tail);
+          tmem_ld_wait();
+        }
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 32) {
           uint32_t pk[16];
@@ -330,6 +352,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
+        if (tail_bh >= 0) {
+          float* dst = tail_dst();
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            atomicAdd(reinterpret_cast<float4*>(dst + (c / 4) * (kT * 4)),
+                      make_float4(__uint_as_float(tail[c]), __uint_as_float(tail[c + 1]),
+                                  __uint_as_float(tail[c + 2]), __uint_as_float(tail[c + 3])));
+          tail_bh = -1;
+        }
         // dS^T = P^T (dP^T - D) -> bf16 rows of 64 queries, 128-byte swizzle,
         // into the X buffer (dO there has been read: dp_full follows dV)
         if (!(ok = mbar_wait(dp_full, nv & 1, a.ctx, abort_flag))) break;
@@ -357,25 +388,28 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(ds_full);
-        // dQ of the visit: this half's 96 columns of query `row`, added into
-        // the workspace with 16-byte reductions (a warp: 512 contiguous bytes)
+        // dQ of the visit (query `row`): the 64 columns the next S^T will
+        // overwrite now, added into the workspace with 16-byte reductions (a
+        // warp: 512 contiguous bytes); the other 32 at the next visit
         if (!(ok = mbar_wait(dq_full, nv & 1, a.ctx, abort_flag))) break;
         tc_fence_after();
         {
-          float acc[kDQK / 2];
-#pragma unroll
-          for (int c0 = 0; c0 < kDQK / 2; c0 += 32) tmem_ld32f(lb + C::DQ + dc + c0, acc + c0);
+          float acc[64];
+          tmem_ld32f(lb + C::DQ + dqa, acc);
+          tmem_ld32f(lb + C::DQ + dqa + 32, acc + 32);
           tmem_ld_wait();
-#pragma unroll
-          for (int c0 = 0; c0 < kDQK / 2; c0 += 32) reg_fence32(acc + c0);
+          reg_fence32(acc);
+          reg_fence32(acc + 32);
           tc_fence_before();
           mbar_arrive(dq_empty);
-          float* dst = a.ws_dq + bwd_dq_index(a, it.b * a.Hq + h, qt * kT + row, dc, kDQK);
+          float* dst = a.ws_dq + bwd_dq_index(a, it.b * a.Hq + h, qt * kT + row, dqa, kDQK);
 #pragma unroll
-          for (int c = 0; c < kDQK / 2; c += 4)
+          for (int c = 0; c < 64; c += 4)
             atomicAdd(reinterpret_cast<float4*>(dst + (c / 4) * (kT * 4)),
                       make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
         }
+        tail_bh = it.b * a.Hq + h;
+        tail_qt = qt;
         ++nv;
         any = true;
       }
@@ -396,6 +430,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
         mbar_arrive(acc_empty);
         ++nacc;
       }
+    }
+    // the last visit's remaining dQ columns (its dq_full was waited above)
+    if (ok && tail_bh >= 0) {
+      float tail[32];
+      tc_fence_after();
+      tmem_ld32f(lb + C::DQ + dqb, tail);
+      tmem_ld_wait();
+      reg_fence32(tail);
+      float* dst = tail_dst();
+#pragma unroll
+      for (int c = 0; c < 32; c += 4)
+        atomicAdd(reinterpret_cast<float4*>(dst + (c / 4) * (kT * 4)),
+                  make_float4(tail[c], tail[c + 1], tail[c + 2], tail[c + 3]));
     }
   }
 
