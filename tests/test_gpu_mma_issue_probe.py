@@ -1,8 +1,10 @@
 """GPU check of a property of the hardware that the kernels' MMA-issue design
-relies on (DESIGN: measured forward findings): one warp can keep the tensor
-pipe busy with M = 128, K = 16 tcgen05.mma instructions -- 64 cycles each at
-N = 128, 128 at N = 256 -- when it forms the operand descriptors as a
-converged warp and one elected lane issues.  The probe (tests/probes/
+relies on: one warp can keep the tensor pipe busy with M = 128, K = 16
+tcgen05.mma instructions -- 64 cycles each at N = 128, 128 at N = 256 --
+when it forms the operand descriptors as a converged warp and one elected
+lane issues.  (In the attention kernels, where the issuing warp shares its
+sub-partition with busy softmax warps, that form measured slower than one
+lane issuing alone, so the kernels keep the latter.)  The probe (tests/probes/
 mma_issue_probe.cu, built here with nvcc against the library's PTX wrappers)
 also reports the lane-0 forms the kernels use, for the record."""
 import json
