@@ -21,7 +21,11 @@ __device__ __forceinline__ bool elect_lane() {
   return pred != 0;
 }
 
-__global__ void __launch_bounds__(128, 1) probe(int mode, long long* out, int* err) {
+// Each form is its own instantiation (MODE), so that the code the compiler
+// generates for one does not depend on the others.
+template <int MODE>
+__global__ void __launch_bounds__(128, 1) probe(long long* out, int* err) {
+  constexpr int mode = MODE;
   extern __shared__ uint8_t raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   uint8_t* A = sm;               // 128 rows x 128 bf16: 2 atoms of 16 KB
@@ -45,8 +49,8 @@ __global__ void __launch_bounds__(128, 1) probe(int mode, long long* out, int* e
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t a_base = smem_u32(A), b_base = smem_u32(B);
-  const uint32_t id = idesc_bf16_f32(128, mode == 3 ? 256 : 128, 0, 0);
-  const bool converged = mode == 1;
+  constexpr uint32_t id = idesc_bf16_f32(128, mode == 3 ? 256 : 128, 0, 0);
+  constexpr bool converged = mode == 1;
   if (warp == 0 && (converged || lane == 0)) {
     const uint64_t da = sdesc_k_sw128(a_base);
     const long long t0 = clock64();
@@ -54,7 +58,7 @@ __global__ void __launch_bounds__(128, 1) probe(int mode, long long* out, int* e
       const int s = bt % 3;
       const uint64_t db = sdesc_k_sw128(b_base + s * 65536);
       const uint32_t d = tmem + (bt & 1) * 256;
-      if (mode == 2) {  // descriptors formed first, then issued
+      if constexpr (mode == 2) {  // descriptors formed first, then issued
         uint64_t pa[8], pb[8];
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -69,8 +73,12 @@ __global__ void __launch_bounds__(128, 1) probe(int mode, long long* out, int* e
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
           const uint32_t offb = ((ks >> 2) * 32768 + (ks & 3) * 32) >> 4;
-          if (!converged || elect_lane()) umma_ss(d, da + off, db + offb, id, ks > 0 ? 1u : 0u);
-          if (converged) __syncwarp();
+          if constexpr (converged) {
+            if (elect_lane()) umma_ss(d, da + off, db + offb, id, ks > 0 ? 1u : 0u);
+            __syncwarp();
+          } else {
+            umma_ss(d, da + off, db + offb, id, ks > 0 ? 1u : 0u);
+          }
         }
       }
     }
@@ -90,6 +98,19 @@ __global__ void __launch_bounds__(128, 1) probe(int mode, long long* out, int* e
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+template <int MODE>
+bool run(int sms, int smem, long long* d_out, int* d_err, double* cyc) {
+  cudaFuncSetAttribute(probe<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  for (int rep = 0; rep < 3; ++rep) probe<MODE><<<sms, 128, smem>>>(d_out, d_err);
+  if (cudaDeviceSynchronize() != cudaSuccess) return false;
+  std::vector<long long> h(sms);
+  cudaMemcpy(h.data(), d_out, sms * sizeof(long long), cudaMemcpyDeviceToHost);
+  double s = 0;
+  for (long long x : h) s += static_cast<double>(x);
+  *cyc = s / sms / (kBatches * 8);
+  return true;
+}
+
 int main() {
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, 0) != cudaSuccess) return 2;
@@ -100,20 +121,13 @@ int main() {
   cudaMemset(d_err, 0, sizeof(int));
   const int smem = 1024 + 32768 + 3 * 65536 + 1024;
   if (smem > 232448) return 3;
-  cudaFuncSetAttribute(probe, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  const char* names[kModes] = {"lane0_inline", "converged_elect", "lane0_formed_first", "lane0_inline_n256"};
-  printf("{");
-  for (int mode = 0; mode < kModes; ++mode) {
-    for (int rep = 0; rep < 3; ++rep) probe<<<sms, 128, smem>>>(mode, d_out, d_err);
-    if (cudaDeviceSynchronize() != cudaSuccess) return 4;
-    std::vector<long long> h(sms);
-    cudaMemcpy(h.data(), d_out, sms * sizeof(long long), cudaMemcpyDeviceToHost);
-    double s = 0;
-    for (long long x : h) s += static_cast<double>(x);
-    printf("%s\"%s\": %.1f", mode ? ", " : "", names[mode], s / sms / (kBatches * 8));
-  }
+  double c[kModes];
+  if (!run<0>(sms, smem, d_out, d_err, &c[0]) || !run<1>(sms, smem, d_out, d_err, &c[1]) ||
+      !run<2>(sms, smem, d_out, d_err, &c[2]) || !run<3>(sms, smem, d_out, d_err, &c[3]))
+    return 4;
   int herr = 0;
   cudaMemcpy(&herr, d_err, sizeof(int), cudaMemcpyDeviceToHost);
-  printf(", \"timeouts\": %d}\n", herr);
+  printf("{\"lane0_inline\": %.1f, \"converged_elect\": %.1f, \"lane0_formed_first\": %.1f, "
+         "\"lane0_inline_n256\": %.1f, \"timeouts\": %d}\n", c[0], c[1], c[2], c[3], herr);
   return herr ? 5 : 0;
 }
