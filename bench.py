@@ -262,37 +262,45 @@ def run_ours(args, world, rank):
                          "peak_kind": f"fp32 FMA: {num_sms} SMs x 128 lanes x 2 FLOP x {mhz} MHz",
                          "frac_of_sustained": None})
 
-    # end to end through the public API from pinned host buffers: every step
-    # copies its inputs in and its output and LSE out, inside the timed
-    # region; the pipeline overlaps one step's copies with its neighbours'
-    # kernels (two device buffer sets, separate copy and compute streams)
-    from ring_context_parallelism_ra_b200.host_pipeline import RingForwardPipeline
+    # end to end through the C ABI on host buffers: every step is one
+    # ra_ring_forward_host call (Q, K, V copied in from pinned host memory,
+    # the ring, O and LSE copied back), the copies of one chunk of heads
+    # overlapping the kernels of its neighbours inside the call
     qh = q.cpu().pin_memory()
     kh = k.cpu().pin_memory()
     vh = v.cpu().pin_memory()
-    pipe = RingForwardPipeline(q.shape, k.shape, v.shape, q.dtype, wl.P, wl.causal, wl.scale)
+    del q, k, v, out, lse
+    torch.cuda.empty_cache()
+    out_h = torch.empty((wl.B, wl.Hq, wl.n, wl.d_v), dtype=wl.torch_dtype, pin_memory=True)
+    lse_h = torch.empty((wl.B, wl.Hq, wl.n), dtype=torch.float32, pin_memory=True)
+    ws = torch.empty(ra.ring_forward_host_workspace_bytes(qh, kh, vh), dtype=torch.uint8,
+                     device=dev)
+
+    def host_step():
+        ra.ring_forward_host(qh, kh, vh, wl.P, wl.causal, wl.scale, out_h, lse_h, ws,
+                             stream=stream, synchronize=False)
+
     for _ in range(3):
-        pipe.wait(pipe.submit(qh, kh, vh))
+        host_step()
+    torch.cuda.synchronize()
     e2e_steps = max(3, min(args.steps, 20))
     barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(pipe.s_in)
+    e0.record(stream)
     for _ in range(e2e_steps):
-        pipe.submit(qh, kh, vh)
-    pipe.drain_on(stream)
+        host_step()
     e1.record(stream)
     torch.cuda.synchronize()
+    assert ra.get_status() == ra.RA_OK
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
-    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
     e2e = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
-           "api": "RingForwardPipeline (ring_forward per step; copies of a step overlap "
-                  "its neighbours' kernels)"}
-    bufs = None
-    del qh, kh, vh, bufs, pipe, q, k, v, out, lse, flush
+           "api": "ra_ring_forward_host (one C-ABI call per step: copies in, ring, copies out)"}
+    del qh, kh, vh, out_h, lse_h, ws, flush
     torch.cuda.empty_cache()
 
     decode = None if args.skip_decode else run_decode_leg(args, world, rank, peaks, peaks_kind)

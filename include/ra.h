@@ -153,6 +153,49 @@ int ra_ring_forward_striped(const void* q, const void* k, const void* v, int P, 
                             void* stream);
 
 /*
+ * ra_ring_forward_host_workspace_bytes -- device bytes ra_ring_forward_host
+ * needs for `shape` (two chunk buffer sets).  A pure function of the shape;
+ * 0 for an invalid shape.
+ */
+size_t ra_ring_forward_host_workspace_bytes(const ra_shape* shape);
+
+/*
+ * ra_ring_forward_host -- ra_ring_forward (the same fused ring, the same
+ * result) on tensors in HOST memory: the inputs are copied in, the ring runs,
+ * O and LSE are copied out, all enqueued by this one call.  The (batch, KV
+ * head) groups are processed in up to 8 equal chunks of whole groups (a
+ * chunk keeps at least 1024 work items of 256 query rows, else the call uses
+ * fewer chunks, down to one): chunk c's host-to-device copies run on an
+ * internal copy stream while chunk c-1's kernel runs on `stream` and chunk
+ * c-2's results return on a second internal copy stream, through two buffer
+ * sets that alternate in `workspace`.
+ *   q, k, v     : host BHSD as ra_ring_forward (n_q == n_k, n % P == 0).
+ *                 Page-locked (pinned) memory lets the copies overlap the
+ *                 kernels; pageable memory works, but each copy then holds
+ *                 the calling thread until it is done.
+ *   out         : host [B, Hq, n, d_v], same dtype as q.
+ *   lse         : host fp32 [B, Hq, n], or NULL to skip.
+ *   workspace   : device, 256-byte aligned, at least
+ *                 ra_ring_forward_host_workspace_bytes(shape) bytes, owned
+ *                 by the caller and not used by other work until `stream`
+ *                 has passed this call.
+ *   stream      : the kernels run on it; the copies start after the work
+ *                 already on it, and work enqueued on it later starts only
+ *                 after every output byte is in host memory.  The call
+ *                 returns after enqueueing: synchronise `stream` before
+ *                 reading out / lse or writing q, k, v.
+ * The copy streams and their events are created once per device on first
+ * use (released by ra_shutdown); concurrent calls on one device are
+ * enqueued one after another.  No device memory is allocated.
+ * Errors: RA_ERR_INVALID (null, shape, workspace too small or misaligned),
+ * RA_ERR_UNSUPPORTED (head dims), RA_ERR_CUDA (a copy, event or launch
+ * failed; work enqueued before the failure still runs).
+ */
+int ra_ring_forward_host(const void* q, const void* k, const void* v, int P, int causal,
+                         float scale, void* out, float* lse, const ra_shape* shape,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * ra_decode_workspace_bytes -- bytes of device workspace ra_decode_partial
  * needs for `shape` (its split-KV chunk partials).  0 on invalid shape.
  */
@@ -387,7 +430,8 @@ const char* ra_status_string(int status);
 /* Number of kernel launches this library has enqueued since load. */
 unsigned long long ra_launch_count(void);
 
-/* Release cached descriptors.  Safe to call more than once. */
+/* Release cached descriptors and the copy streams / events of
+ * ra_ring_forward_host.  Safe to call more than once. */
 int ra_shutdown(void);
 
 #ifdef __cplusplus

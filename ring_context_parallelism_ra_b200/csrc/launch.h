@@ -14,6 +14,9 @@ namespace ra {
 // Counts kernel launches enqueued by this library (ra_launch_count).
 void note_launch();
 
+// Releases the copy streams and events of ra_ring_forward_host (ra_shutdown).
+void release_host_call_state();
+
 // Per-device state: SM count, status word address, wait bound.
 struct DeviceInfo {
   int device;

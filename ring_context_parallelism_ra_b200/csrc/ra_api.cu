@@ -465,6 +465,7 @@ const char* ra_status_string(int status) {
 unsigned long long ra_launch_count(void) { return g_launches.load(); }
 
 int ra_shutdown(void) {
+  release_host_call_state();
   std::lock_guard<std::mutex> lock(g_dev_mu);
   for (int i = 0; i < kMaxDevices; ++i) g_dev_ready[i] = false;
   return RA_OK;

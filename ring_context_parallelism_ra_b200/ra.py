@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "RAError", "library_path", "lib", "Shape", "block_partial", "block_partial_strided",
     "lse_merge", "ring_forward", "ring_forward_striped",
-    "ring_forward_host", "decode_workspace_bytes", "decode_partial", "decode_partials",
+    "ring_forward_host", "ring_forward_host_workspace_bytes", "decode_workspace_bytes", "decode_partial", "decode_partials",
     "decode_partial_noalloc",
     "decode_merge",
     "decode_pass_q", "backward_workspace_bytes", "backward_delta", "ring_backward",
@@ -34,7 +34,8 @@ RA_F32, RA_BF16 = 0, 1
 # Every symbol include/ra.h declares.
 EXPORTED = (
     "ra_block_partial", "ra_block_partial_strided", "ra_lse_merge", "ra_ring_forward",
-    "ra_ring_forward_striped", "ra_decode_workspace_bytes",
+    "ra_ring_forward_striped", "ra_ring_forward_host_workspace_bytes", "ra_ring_forward_host",
+    "ra_decode_workspace_bytes",
     "ra_decode_partial", "ra_decode_partials", "ra_decode_partial_noalloc", "ra_decode_merge",
     "ra_backward_workspace_bytes", "ra_backward_delta", "ra_ring_backward",
     "ra_ring_backward_striped", "ra_block_backward", "ra_block_class", "ra_block_class_device",
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
             "ra_ring_forward_striped": (i, [vp, vp, vp, i, i, f, vp, vp, sp, vp]),
             "ra_lse_merge": (i, [vp, vp, i, sp, vp, i, vp, vp]),
             "ra_ring_forward": (i, [vp, vp, vp, i, i, f, vp, vp, sp, vp]),
+            "ra_ring_forward_host_workspace_bytes": (sz, [sp]),
+            "ra_ring_forward_host": (i, [vp, vp, vp, i, i, f, vp, vp, sp, vp, sz, vp]),
             "ra_decode_workspace_bytes": (sz, [sp]),
             "ra_decode_partial": (i, [vp, vp, vp, ctypes.c_longlong, sp, f, vp, vp, vp, sz, vp]),
             "ra_decode_partial_noalloc": (i, [vp, vp, vp, ctypes.c_longlong, sp, f, vp, vp, vp]),
@@ -239,25 +242,50 @@ def ring_forward_striped(q, k, v, P, causal=True, scale=None, out=None, lse=None
     return out, lse
 
 
-def ring_forward_host(q, k, v, P, causal=True, scale=None, device="cuda", bufs=None):
-    """End-to-end call from host tensors (pinned for overlap): copy in, run the
-    fused ring, copy O and LSE back.  ``bufs`` may carry preallocated device
-    tensors (q, k, v, out, lse) and pinned host outputs (out_h, lse_h)."""
-    if bufs is None:
-        bufs = {}
-    dq = bufs.get("q") if "q" in bufs else torch.empty(q.shape, dtype=q.dtype, device=device)
-    dk = bufs.get("k") if "k" in bufs else torch.empty(k.shape, dtype=k.dtype, device=device)
-    dv = bufs.get("v") if "v" in bufs else torch.empty(v.shape, dtype=v.dtype, device=device)
-    dq.copy_(q, non_blocking=True)
-    dk.copy_(k, non_blocking=True)
-    dv.copy_(v, non_blocking=True)
-    out, lse = ring_forward(dq, dk, dv, P, causal, scale, bufs.get("out"), bufs.get("lse"))
-    out_h = bufs.get("out_h") if "out_h" in bufs else torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    lse_h = bufs.get("lse_h") if "lse_h" in bufs else torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    out_h.copy_(out, non_blocking=True)
-    lse_h.copy_(lse, non_blocking=True)
-    torch.cuda.current_stream().synchronize()
-    return out_h, lse_h
+def _host(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise TypeError(f"{name} must be a CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def ring_forward_host_workspace_bytes(q, k, v) -> int:
+    """Device bytes ``ring_forward_host`` needs for these shapes."""
+    s = _shape(q, k, v)
+    return int(lib().ra_ring_forward_host_workspace_bytes(ctypes.byref(s)))
+
+
+def ring_forward_host(q, k, v, P, causal=True, scale=None, out=None, lse=None, workspace=None,
+                      stream=None, synchronize=True):
+    """``ra_ring_forward_host``: the fused ring on host tensors (pinned memory
+    for overlapped copies).  Returns (O, LSE) as host tensors (pinned when
+    allocated here); they hold the result once ``stream`` has passed the
+    call, which this wrapper waits for unless ``synchronize`` is False."""
+    s = _shape(q, k, v)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    if out is None:
+        out = torch.empty((s.B, s.Hq, s.n_q, s.d_v), dtype=q.dtype, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((s.B, s.Hq, s.n_q), dtype=torch.float32, pin_memory=True)
+    need = ring_forward_host_workspace_bytes(q, k, v)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    if not workspace.is_cuda:
+        raise TypeError("workspace must be a CUDA tensor")
+    st = stream if stream is not None else torch.cuda.current_stream()
+    rc = lib().ra_ring_forward_host(_host(q, "q"), _host(k, "k", q.dtype), _host(v, "v", q.dtype),
+                                    int(P), int(bool(causal)), float(scale),
+                                    _host(out, "out", q.dtype), _host(lse, "lse", torch.float32),
+                                    ctypes.byref(s), ctypes.c_void_p(workspace.data_ptr()),
+                                    ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                    ctypes.c_void_p(st.cuda_stream))
+    _check("ra_ring_forward_host", rc)
+    if synchronize:
+        st.synchronize()
+    return out, lse
 
 
 def backward_workspace_bytes(q, k, v) -> int:

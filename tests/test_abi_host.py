@@ -207,3 +207,60 @@ def test_decode_graph_rejects_uneven_shards_before_any_gpu_work():
     k = torch.zeros((1, 1, 1000, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="equal shards"):
         PassQDecodeGraph(k, k, 3, 8)
+
+
+def _host_slot_bytes(B, Hq, Hkv, n, dqk, dv, esz, per_chunk):
+    """One chunk buffer set as ra.h describes it: Q, K, V, O, LSE of
+    `per_chunk` (batch, KV head) groups, each buffer 256-byte aligned."""
+    G = Hq // Hkv
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    parts = [G * n * dqk * esz, n * dqk * esz, n * dv * esz, G * n * dv * esz, G * n * 4]
+    return sum(al(per_chunk * b) for b in parts)
+
+
+@pytest.mark.parametrize("dims,per_chunk", [
+    ((1, 16, 16, 262144, 192, 128), 2),   # 1024 items per group: 8 chunks of 2 groups
+    ((1, 32, 8, 131072, 128, 128), 1),    # 2048 items per group: 8 chunks of 1
+    ((1, 8, 8, 8192, 128, 128), 8),       # 32 items per group: one chunk
+    ((8, 2, 2, 32768, 128, 128), 8),      # 128 per group: chunks of 4 whole batches
+    ((2, 8, 2, 65536, 128, 128), 1),      # 1024 per group: 4 chunks (within a batch)
+    ((3, 1, 1, 1000, 64, 64), 3),         # nothing splits: one chunk
+])
+def test_host_call_workspace_follows_the_chunk_rule(dims, per_chunk):
+    B, Hq, Hkv, n, dqk, dv = dims
+    s = _shape(B=B, Hq=Hq, Hkv=Hkv, n_q=n, n_k=n, d_qk=dqk, d_v=dv)
+    want = 2 * _host_slot_bytes(B, Hq, Hkv, n, dqk, dv, 2, per_chunk)
+    assert ra.lib().ra_ring_forward_host_workspace_bytes(ctypes.byref(s)) == want
+    s32 = _shape(B=B, Hq=Hq, Hkv=Hkv, n_q=n, n_k=n, d_qk=dqk, d_v=dv, dtype=ra.RA_F32)
+    want32 = 2 * _host_slot_bytes(B, Hq, Hkv, n, dqk, dv, 4, per_chunk)
+    assert ra.lib().ra_ring_forward_host_workspace_bytes(ctypes.byref(s32)) == want32
+
+
+def test_host_call_rejects_bad_arguments_before_any_gpu_work():
+    L = ra.lib()
+    p = ctypes.c_void_p(256)   # never dereferenced on these paths
+    nul = ctypes.c_void_p(0)
+    INV, UNS = ra.RA_ERR_INVALID, ra.RA_ERR_UNSUPPORTED
+    s = _shape()
+    ws = L.ra_ring_forward_host_workspace_bytes(ctypes.byref(s))
+    assert ws > 0
+    big = ctypes.c_size_t(ws)
+
+    def call(shape=s, P=1, causal=1, q=p, w=p, wsb=big):
+        return L.ra_ring_forward_host(q, p, p, P, causal, 1.0, p, p, ctypes.byref(shape), w,
+                                      wsb, nul)
+
+    assert call(q=nul) == INV
+    assert call(w=nul) == INV
+    assert call(w=ctypes.c_void_p(256 + 16)) == INV          # workspace not 256-byte aligned
+    assert call(wsb=ctypes.c_size_t(ws - 1)) == INV          # workspace too small
+    assert call(P=0) == INV
+    assert call(P=3) == INV                                  # 128 % 3
+    assert call(causal=2) == INV
+    assert call(shape=_shape(n_k=64)) == INV                 # n_q != n_k
+    assert call(shape=_shape(Hq=3, Hkv=2)) == INV
+    assert call(shape=_shape(n_q=0, n_k=0)) == INV
+    wide = _shape(d_qk=96)
+    assert call(shape=wide, wsb=ctypes.c_size_t(1 << 40)) == UNS
+    assert L.ra_ring_forward_host_workspace_bytes(None) == 0
+    assert L.ra_ring_forward_host_workspace_bytes(ctypes.byref(_shape(Hq=3, Hkv=2))) == 0
