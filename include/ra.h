@@ -313,7 +313,8 @@ int ra_decode_merge(const float* o_parts, const float* lse_parts, int P, const r
 /*
  * ra_backward_workspace_bytes -- device workspace the backward calls need for
  * `shape` (an fp32 dQ accumulator and two row vectors, padded to 128 rows
- * per head): about B * Hq * n_q * (d_qk + 2) * 4 bytes.  0 on invalid shape.
+ * per head, and the counter the tensor-core kernels hand out work items
+ * from): about B * Hq * n_q * (d_qk + 2) * 4 bytes.  0 on invalid shape.
  */
 size_t ra_backward_workspace_bytes(const ra_shape* shape);
 

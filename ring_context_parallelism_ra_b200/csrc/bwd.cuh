@@ -32,10 +32,11 @@ constexpr int kBwdTile = 128;  // rows of a dQ workspace tile
 //   nl2  [B*Hq][ntq*128]          -LSE * log2(e) (-inf for a row with no key
 //                                 and for padding rows)
 //   D    [B*Hq][ntq*128]          rowsum(dO * O) (0 for padding rows)
+//   ctr  one 32-bit counter: work items handed out so far (zeroed with dQ)
 struct BwdLayout {
   int ntq;
   long long rows_pad;
-  size_t dq_off, nl2_off, d_off, total;
+  size_t dq_off, nl2_off, d_off, ctr_off, total;
 };
 
 inline size_t bwd_align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -47,7 +48,8 @@ inline BwdLayout bwd_layout(int B, int Hq, int n_q, int d_qk) {
   L.dq_off = 0;
   L.nl2_off = bwd_align256(L.dq_off + static_cast<size_t>(L.rows_pad) * d_qk * 4);
   L.d_off = bwd_align256(L.nl2_off + static_cast<size_t>(L.rows_pad) * 4);
-  L.total = bwd_align256(L.d_off + static_cast<size_t>(L.rows_pad) * 4);
+  L.ctr_off = bwd_align256(L.d_off + static_cast<size_t>(L.rows_pad) * 4);
+  L.total = L.ctr_off + 256;
   return L;
 }
 
@@ -68,6 +70,7 @@ struct BwdArgs {
   void* dk;          // ring: [B, Hkv, n_k, d_qk] of the input dtype; block: fp32, +=
   void* dv;
   int block_mode;
+  unsigned int* item_counter;  // items handed out so far (tensor-core kernels)
   DevCtx ctx;
 };
 
@@ -83,18 +86,14 @@ struct BItem {
   long long koff;  // key position = koff + key index * stride
 };
 
-// Items are dealt in snake order over the persistent CTAs, heaviest first for
-// a causal mask: low key positions are visible to the most queries.  They
-// come in blocks of kv_block (batch, KV head)s whose dQ accumulator fits in
-// L2 (all of a block's items before the next block's): the CTAs that run at
-// the same time then walk the same query tiles and add their dQ shares into
-// the same lines of L2, instead of spreading the reductions over a workspace
-// far larger than L2.
-__device__ __forceinline__ bool bwd_item_at(const BwdArgs& a, int round, BItem& it) {
-  const int nc = gridDim.x;
-  const int c = blockIdx.x;
-  const long long idx = static_cast<long long>(round) * nc + ((round & 1) ? (nc - 1 - c) : c);
-  if (idx >= a.items) return false;
+// Item `idx` in the order work is handed out, heaviest first for a causal
+// mask: low key positions are visible to the most queries.  Items come in
+// blocks of kv_block (batch, KV head)s whose dQ accumulator fits in L2 (all
+// of a block's items before the next block's), so that the CTAs running at
+// the same time walk the same query tiles and add their dQ shares into the
+// same lines of L2 instead of spreading the reductions over a workspace far
+// larger than L2.
+__device__ __forceinline__ void bwd_item_from_index(const BwdArgs& a, long long idx, BItem& it) {
   const int nbkv = a.B * a.Hkv;
   const int blk = static_cast<int>(idx / (static_cast<long long>(a.ntk) * a.kv_block));
   const int kv0 = blk * a.kv_block;
@@ -116,6 +115,16 @@ __device__ __forceinline__ bool bwd_item_at(const BwdArgs& a, int round, BItem& 
   const int j = it.k0 / Lk;
   it.j = j < a.P - 1 ? j : a.P - 1;
   it.koff = bwd_part_offset(a, it.j, a.n_k, a.k_offset);
+}
+
+// Static dealing (one item per CTA and round, snake order over the CTAs),
+// for the kernels launched with one CTA per item.
+__device__ __forceinline__ bool bwd_item_at(const BwdArgs& a, int round, BItem& it) {
+  const int nc = gridDim.x;
+  const int c = blockIdx.x;
+  const long long idx = static_cast<long long>(round) * nc + ((round & 1) ? (nc - 1 - c) : c);
+  if (idx >= a.items) return false;
+  bwd_item_from_index(a, idx, it);
   return true;
 }
 

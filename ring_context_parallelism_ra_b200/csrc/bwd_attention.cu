@@ -129,7 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
   uint64_t* drain = bars + 14;
   uint64_t* s_read = bars + 15;  // both compute halves hold their S^T
   uint64_t* dk_done = bars + 16;  // dK(v) has read the dS tile
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  const ItemQueue iq{reinterpret_cast<volatile int*>(bars + 17 + 2 * kItemSlots), bars + 17,
+                     bars + 17 + kItemSlots};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17 + 2 * kItemSlots + kItemSlots / 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* kv_issued = abort_flag + 1;
   volatile int* q_issued = abort_flag + 2;
@@ -155,6 +157,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
     mbar_init(drain, 3);
     mbar_init(s_read, 2 * kT);
     mbar_init(dk_done, 1);
+    for (int i = 0; i < kItemSlots; ++i) {
+      mbar_init(&iq.full[i], 1);
+      mbar_init(&iq.empty[i], 3 + 2 * kT);  // the three issuers, the compute threads
+    }
     *abort_flag = 0;
     *kv_issued = 0;
     *q_issued = 0;
@@ -180,7 +186,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
       uint32_t nkv = 0, nq = 0;
       BItem it;
       bool ok = true;
-      for (int round = 0; ok && !*abort_flag && bwd_item_at(a, round, it); ++round) {
+      for (int round = 0; ok && !*abort_flag; ++round) {
+        const int idx = item_publish(iq, a.item_counter, a.items, round, a.ctx, abort_flag);
+        if (idx < 0) {
+          ok = idx == -1;
+          break;
+        }
+        bwd_item_from_index(a, idx, it);
         QWalk w;
         w.start(a, it);
         int qt, h;
@@ -225,7 +237,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
       uint32_t nkv = 0, nv = 0, nacc = 0;  // nv: visits so far = query-stage counter
       BItem it;
       bool ok = true;
-      for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
+      for (int round = 0; ok; ++round) {
+        const int idx = item_take(iq, round, a.ctx, abort_flag);
+        if (idx < 0) {
+          ok = idx == -1;
+          break;
+        }
+        bwd_item_from_index(a, idx, it);
         QWalk w;
         w.start(a, it);
         int qt, h;
@@ -349,7 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(
                   make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
       return true;
     };
-    for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
+    for (int round = 0; ok; ++round) {
+      const int idx = item_take(iq, round, a.ctx, abort_flag);
+      if (idx < 0) {
+        ok = idx == -1;
+        break;
+      }
+      bwd_item_from_index(a, idx, it);
       QWalk w;
       w.start(a, it);
       int qt, h;
@@ -515,7 +539,8 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
   float* ws_d = reinterpret_cast<float*>(ws + L.d_off);
 
   int rc = launch_backward_rows(block_mode ? nullptr : out, dout, delta, lse, s, L, ws_nl2, ws_d,
-                                ws_dq, dev, stream);
+                                ws_dq, reinterpret_cast<unsigned int*>(ws + L.ctr_off), dev,
+                                stream);
   if (rc != RA_OK) return rc;
 
   BwdArgs a{};
@@ -540,6 +565,7 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
   a.dk = dk;
   a.dv = dv;
   a.block_mode = block_mode ? 1 : 0;
+  a.item_counter = reinterpret_cast<unsigned int*>(ws + L.ctr_off);
   a.ctx = dev.ctx;
   // as many (batch, KV head)s per block of items as keep the dQ accumulator
   // of their query heads within 48 MB (well inside the 126 MB L2)

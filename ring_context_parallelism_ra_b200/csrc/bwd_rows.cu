@@ -26,6 +26,7 @@ struct PrepArgs {
   float* dq_ws;        // zeroed when non-null
   long long dq_floats;
   float* delta_out;    // [B * Hq * n_q] or null
+  unsigned int* counter;  // backward work-item counter, zeroed when non-null
 };
 
 // Eight consecutive elements of a row as fp32 (one 16-byte load for bf16, two
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(PrepArgs p) {
       if (p.delta_out && t < p.n_q) p.delta_out[bh * p.n_q + t] = dsum;
     }
   }
+  if (p.counter != nullptr && tid == 0) *p.counter = 0u;
   if (p.dq_ws != nullptr) {
     float4* z = reinterpret_cast<float4*>(p.dq_ws);
     const long long n4 = p.dq_floats / 4;
@@ -178,8 +180,10 @@ int launch_backward_delta(const void* out, const void* dout, const ra_shape& s, 
 
 int launch_backward_rows(const void* out, const void* dout, const float* delta, const float* lse,
                          const ra_shape& s, const BwdLayout& L, float* nl2, float* d_ws,
-                         float* dq_ws, const DeviceInfo& dev, cudaStream_t stream) {
+                         float* dq_ws, unsigned int* counter, const DeviceInfo& dev,
+                         cudaStream_t stream) {
   PrepArgs p{};
+  p.counter = counter;
   p.out = out;
   p.dout = dout;
   p.delta = delta;

@@ -125,7 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
   uint64_t* acc_full = bars + 14;
   uint64_t* acc_empty = bars + 15;
   uint64_t* drain = bars + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  const ItemQueue iq{reinterpret_cast<volatile int*>(bars + 17 + 2 * kItemSlots), bars + 17,
+                     bars + 17 + kItemSlots};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17 + 2 * kItemSlots + kItemSlots / 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* kv_issued = abort_flag + 1;
   volatile int* q_issued = abort_flag + 2;
@@ -152,6 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kT);
     mbar_init(drain, 1);
+    for (int i = 0; i < kItemSlots; ++i) {
+      mbar_init(&iq.full[i], 1);
+      mbar_init(&iq.empty[i], 1 + 2 * kT);  // the issuer, the compute threads
+    }
     *abort_flag = 0;
     *kv_issued = 0;
     *q_issued = 0;
@@ -178,7 +184,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
       uint32_t nkv = 0, nq = 0;
       BItem it;
       bool ok = true;
-      for (int round = 0; ok && !*abort_flag && bwd_item_at(a, round, it); ++round) {
+      for (int round = 0; ok && !*abort_flag; ++round) {
+        const int idx = item_publish(iq, a.item_counter, a.items, round, a.ctx, abort_flag);
+        if (idx < 0) {
+          ok = idx == -1;
+          break;
+        }
+        bwd_item_from_index(a, idx, it);
         QWalk w;
         w.start(a, it);
         int qt, h;
@@ -221,7 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
       uint32_t nkv = 0, nv = 0, nacc = 0;
       BItem it;
       bool ok = true;
-      for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
+      for (int round = 0; ok; ++round) {
+        const int idx = item_take(iq, round, a.ctx, abort_flag);
+        if (idx < 0) {
+          ok = idx == -1;
+          break;
+        }
+        bwd_item_from_index(a, idx, it);
         QWalk w;
         w.start(a, it);
         int qt, h;
@@ -297,7 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc192_kernel(
     };
     BItem it;
     bool ok = true;
-    for (int round = 0; ok && bwd_item_at(a, round, it); ++round) {
+    for (int round = 0; ok; ++round) {
+      const int idx = item_take(iq, round, a.ctx, abort_flag);
+      if (idx < 0) {
+        ok = idx == -1;
+        break;
+      }
+      bwd_item_from_index(a, idx, it);
       QWalk w;
       w.start(a, it);
       int qt, h;

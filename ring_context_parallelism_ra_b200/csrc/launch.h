@@ -73,10 +73,12 @@ int launch_backward_delta(const void* out, const void* dout, const ra_shape& s, 
                           const DeviceInfo& dev, cudaStream_t stream);
 struct BwdArgs;
 struct BwdLayout;
-// Row statistics and zeroed dQ accumulator; dQ accumulator -> output.
+// Row statistics, zeroed dQ accumulator and item counter; dQ accumulator ->
+// output.
 int launch_backward_rows(const void* out, const void* dout, const float* delta, const float* lse,
                          const ra_shape& s, const BwdLayout& L, float* nl2, float* d_ws,
-                         float* dq_ws, const DeviceInfo& dev, cudaStream_t stream);
+                         float* dq_ws, unsigned int* counter, const DeviceInfo& dev,
+                         cudaStream_t stream);
 int launch_dq_finalize(const float* ws_dq, void* dq, const ra_shape& s, const BwdLayout& L,
                        float scale, bool block_mode, cudaStream_t stream);
 int launch_simt_backward(const void* q, const void* k, const void* v, const void* dout,
