@@ -531,14 +531,14 @@ def run_backward_leg(args, world, rank, wl, peaks, peaks_kind):
             "clocks": clk.summary()}
 
 
-TC_FILES = ["tc_attention.cu", "ptx.cuh", "block_class.cuh"]
+TC_FILES = ["tc_attention.cu", "item_queue.cuh", "ptx.cuh", "block_class.cuh"]
 # every prefill workload is timed: the headline one in the main leg, the
 # others in the `workloads` leg
 PREFILL_WORKLOADS = ("causal_mla_256k", "causal_gqa_128k", "causal_mha_8k", "noncausal_fp32_512")
 # the backward leg (every bf16 prefill workload; all run on the tensor cores)
 BACKWARD_WORKLOADS = ("causal_mla_256k", "causal_gqa_128k", "causal_mha_8k")
-BWD_FILES = ["bwd_attention.cu", "bwd_tc.cuh", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
-BWD192_FILES = ["bwd_tc192.cu", "bwd_tc.cuh", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
+BWD_FILES = ["bwd_attention.cu", "bwd_tc.cuh", "item_queue.cuh", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
+BWD192_FILES = ["bwd_tc192.cu", "bwd_tc.cuh", "item_queue.cuh", "bwd.cuh", "ptx.cuh", "block_class.cuh"]
 
 
 def run_striped_leg(args, world, rank, wl, peaks):

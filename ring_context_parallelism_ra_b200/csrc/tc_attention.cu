@@ -26,8 +26,9 @@
 // launch allocation would never proceed; the launcher checks the compiled
 // register count against the split before every launch.)
 // Work item = 256 query rows (two 128-row tiles) of one (batch, head); items
-// are dealt in blocks of KV heads whose K/V fit in L2, heaviest first within
-// a block, in snake order across the persistent CTAs.
+// come in blocks of KV heads whose K/V fit in L2, heaviest first within a
+// block, and the producer of each persistent CTA takes the next one from a
+// global counter.
 //
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [  0,128) S0 = Q0 K^T   (P0 as packed bf16 over its first 64 columns)
@@ -42,8 +43,12 @@
 // max keeps p <= 256; the final division by l makes the result exact).
 #include <cuda.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "block_class.cuh"
 #include "common.cuh"
+#include "item_queue.cuh"
 #include "launch.h"
 #include "ptx.cuh"
 #include "tmap.h"
@@ -96,7 +101,8 @@ struct TcArgs {
   float* lse;         // [B*Hq, n_q] or null
   int n_pairs, items;
   int Lq, Lk;         // rows / keys per partition (n_q / P, n_k / P)
-  int kv_block;       // (batch, KV head)s per block of items (see item_at)
+  int kv_block;       // (batch, KV head)s per block of items (see item_from_index)
+  unsigned int* item_counter;  // items handed out so far (zeroed before the launch)
   DevCtx ctx;
 };
 
@@ -118,15 +124,12 @@ __device__ __forceinline__ long long part_offset(const TcArgs& a, int p, int len
                    : static_cast<long long>(base);
 }
 
-__device__ __forceinline__ bool item_at(const TcArgs& a, int round, Item& it) {
-  const int nc = gridDim.x;
-  const int c = blockIdx.x;
-  const long long idx = static_cast<long long>(round) * nc + ((round & 1) ? (nc - 1 - c) : c);
-  if (idx >= a.items) return false;
-  // Items are dealt in blocks of kv_block (batch, KV head)s whose K and V
-  // fit in L2 together: every item of a block -- heaviest pairs first, the
-  // query heads of the block next to each other -- before the next block's,
-  // so the CTAs that run at the same time stream the same K/V tiles.
+// Item `idx` in the order work is handed out (from a global counter, see
+// item_queue.cuh): blocks of kv_block (batch, KV head)s whose K and V fit in
+// L2 together, every item of a block -- heaviest pairs first, the query heads
+// of the block next to each other -- before the next block's, so the CTAs
+// that run at the same time stream the same K/V tiles.
+__device__ __forceinline__ void item_from_index(const TcArgs& a, long long idx, Item& it) {
   const int G = a.Hq / a.Hkv;
   const int n_kv = a.B * a.Hkv;
   const long long per_kv = static_cast<long long>(a.n_pairs) * G;
@@ -160,7 +163,6 @@ __device__ __forceinline__ bool item_at(const TcArgs& a, int round, Item& it) {
   const int i = it.q0[0] / a.Lq;
   it.i = i < a.P - 1 ? i : a.P - 1;
   it.qoff = part_offset(a, it.i, a.Lq, a.q_offset);
-  return true;
 }
 
 // The KV tiles an item visits, in ring order; every role runs this same walk.
@@ -326,13 +328,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* drain = o_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* iq_full = drain + 1;               // [kItemSlots]
+  uint64_t* iq_empty = iq_full + kItemSlots;   // [kItemSlots]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(iq_empty + kItemSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* kv_issued = abort_flag + 1;
   volatile int* q_issued = abort_flag + 2;
   volatile uint32_t* item_has_tiles = reinterpret_cast<volatile uint32_t*>(abort_flag + 3);
   volatile uint32_t* hdr = item_has_tiles + 1;  // [kNT] headers of K loads
   int* unit_owner = const_cast<int*>(reinterpret_cast<volatile int*>(hdr + kNT));  // [NUNIT]
+  const ItemQueue iq{reinterpret_cast<volatile int*>(unit_owner + NUNIT), iq_full, iq_empty};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -351,6 +356,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
       mbar_init(&o_full[t], 1);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kItemSlots; ++i) {
+      mbar_init(&iq_full[i], 1);
+      mbar_init(&iq_empty[i], 1 + 2 * kBM);  // the MMA thread, the softmax threads
+    }
     *abort_flag = 0;
     *kv_issued = 0;
     *q_issued = 0;
@@ -395,7 +404,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
         }
         return true;
       };
-      for (int round = 0; ok && !*abort_flag && item_at(a, round, it); ++round) {
+      for (int round = 0; ok && !*abort_flag; ++round) {
+        const int idx = item_publish(iq, a.item_counter, a.items, round, a.ctx, abort_flag);
+        if (idx < 0) {
+          ok = idx == -1;
+          break;
+        }
+        item_from_index(a, idx, it);
         if (!mbar_wait(q_empty, (qi & 1) ^ 1, a.ctx, abort_flag)) break;
         TileWalk w;
         w.start(a, it);
@@ -453,7 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
       const uint32_t kv_base = smem_u32(sKV);
       Item it;
       bool ok = true;
-      for (int round = 0; ok && item_at(a, round, it); ++round) {
+      for (int round = 0; ok; ++round) {
+        const int idx = item_take(iq, round, a.ctx, abort_flag);
+        if (idx < 0) {
+          ok = idx == -1;
+          break;
+        }
+        item_from_index(a, idx, it);
         if (!(ok = mbar_wait(q_full, qi & 1, a.ctx, abort_flag))) break;
         ++qi;
         tc_fence_after();
@@ -539,7 +560,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
     uint32_t sph = 0, oph = 0;
     Item it;
     bool ok = true;
-    for (int round = 0; ok && item_at(a, round, it); ++round) {
+    for (int round = 0; ok; ++round) {
+      const int idx = item_take(iq, round, a.ctx, abort_flag);
+      if (idx < 0) {
+        ok = idx == -1;
+        break;
+      }
+      item_from_index(a, idx, it);
       float m = -INFINITY, l = 0.f;
       bool any = false;
       const long long st = pos_stride(a);
@@ -738,6 +765,37 @@ int dispatch(int dqk, int dv, const CUtensorMap& tq, const CUtensorMap& tk, cons
 
 }  // namespace
 
+namespace {
+
+// Work-item counters of the forward launches: a ring of slots in device
+// memory (one array per device); each launch takes the next slot and zeroes
+// it on its stream before the kernel.  Launches that run at the same time on
+// different streams use different slots as long as fewer than kCounterSlots
+// are in flight.
+constexpr int kCounterSlots = 1024;
+__device__ unsigned int g_tc_item_counters[kCounterSlots];
+std::mutex g_ctr_mu;
+unsigned int* g_ctr_base[64] = {};
+std::atomic<unsigned int> g_ctr_next{0};
+
+int item_counter_slot(int device, cudaStream_t stream, unsigned int** out) {
+  if (device < 0 || device >= 64) return RA_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lock(g_ctr_mu);
+    if (g_ctr_base[device] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_tc_item_counters) != cudaSuccess) return RA_ERR_CUDA;
+      g_ctr_base[device] = static_cast<unsigned int*>(p);
+    }
+  }
+  unsigned int* c = g_ctr_base[device] + (g_ctr_next.fetch_add(1) % kCounterSlots);
+  if (cudaMemsetAsync(c, 0, sizeof(unsigned int), stream) != cudaSuccess) return RA_ERR_CUDA;
+  *out = c;
+  return RA_OK;
+}
+
+}  // namespace
+
 int launch_tc_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
                         int q_offset, int k_offset, long long stride, int causal,
                         int striped, float scale, void* out, bool out_f32, float* lse,
@@ -781,6 +839,8 @@ int launch_tc_attention(const void* q, const void* k, const void* v, const ra_sh
   const long long n_kv = static_cast<long long>(s.B) * s.Hkv;
   a.kv_block = static_cast<int>(fit < 1 ? 1 : (fit > n_kv ? n_kv : fit));
   a.ctx = dev.ctx;
+  const int rc = item_counter_slot(dev.device, stream, &a.item_counter);
+  if (rc != RA_OK) return rc;
   const int grid = a.items < dev.num_sms ? a.items : dev.num_sms;
   return out_f32 ? dispatch<true>(s.d_qk, s.d_v, tq, tk, tv, a, grid, stream)
                  : dispatch<false>(s.d_qk, s.d_v, tq, tk, tv, a, grid, stream);
