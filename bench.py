@@ -340,6 +340,27 @@ def run_ours(args, world, rank):
     return line
 
 
+def recap(line):
+    """Every leg's headline figure in a few hundred characters, placed near
+    the end of the line (with the decode leg after it) so that a log that
+    keeps only the line's tail still carries them: value and fraction of the
+    measured peak per prefill and backward workload, end to end, merge."""
+    def short(entry):
+        return [entry["value"], entry["roofline"]["frac"]]
+    r = {"prefill": {line["config"]["workload"]: [line["value"], line["roofline"]["frac"]]},
+         "e2e_tflops": line["e2e"]["value"]}
+    for w in line.get("workloads", []):
+        r["prefill"][w["workload"]] = short(w)
+    if "backward" in line:
+        r["backward"] = {b["workload"]: short(b) for b in line["backward"]}
+    if "merge" in line:
+        r["merge_gbs"] = [m["value"] for m in line["merge"]]
+    if "striped" in line:
+        r["striped_ring_speedup"] = line["striped"].get("ring_speedup_striped_over_contiguous")
+    r["format"] = "workload: [value, fraction of the measured peak]"
+    return r
+
+
 def config_of(wl, world):
     """The line's `config`; both arms print the same dict for a workload."""
     return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "seq_len": wl.n,
@@ -776,6 +797,7 @@ def main():
         val, cores, desc, _ = oracle_sample(workload(args.workload), args.cpu_budget_s)
         line["cpu_baseline"] = {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores,
                                 "kind": "oracle", "sample": desc}
+        line["recap"] = recap(line)
         for key in ("decode_short_cache", "decode"):   # keep the decode leg last
             if key in line:
                 line[key] = line.pop(key)
