@@ -387,14 +387,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(
       int pos = 0;
       Item it;
       bool ok = true;
-      // claim `n` units from `u0` for load L: wait until their previous
-      // loads have been consumed
+      // claim `n` units from `u0` for load L: wait until load L - kNT (the
+      // previous user of L's barriers and header) has been consumed -- the
+      // tensor cores release loads in the order they were issued, so every
+      // older load has been too -- and then for each unit's last load where
+      // that is more recent.  (A unit the ring skips for a while, e.g. one a
+      // contiguous V tile jumps over at the end of the ring, may keep an
+      // owner whose barrier has been reused since.)
       auto claim = [&](int u0, int n, uint32_t L) -> bool {
+        if (L >= static_cast<uint32_t>(kNT) &&
+            !mbar_wait(&ld_empty[L % kNT], ((L - kNT) / kNT) & 1, a.ctx, abort_flag))
+          return false;
         int waited = -1;
         for (int b = 0; b < n; ++b) {
           const int u = u0 + b < NUNIT ? u0 + b : u0 + b - NUNIT;
           const int o = unit_owner[u];
-          if (o >= 0 && o != waited) {
+          if (o >= 0 && static_cast<uint32_t>(o) + kNT > L && o != waited) {
             if (!mbar_wait(&ld_empty[o % kNT], (static_cast<uint32_t>(o) / kNT) & 1, a.ctx,
                            abort_flag))
               return false;
