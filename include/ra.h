@@ -22,7 +22,13 @@
  *     query at q_offset + t iff k_offset + u <= q_offset + t.
  *   - Pointers must be 16-byte aligned.  The library allocates no device
  *     memory per call; what it caches (TMA descriptors, a status word) is
- *     created on first use and released by ra_shutdown().
+ *     created on first use and released by ra_shutdown().  The persistent
+ *     attention kernels take their work items from a counter: the forward
+ *     uses one slot of a module-global ring of 1024 counters per call and
+ *     zeroes it with a 4-byte cudaMemsetAsync on `stream` before the kernel
+ *     (calls running at the same time on different streams get different
+ *     slots while fewer than 1024 are in flight); the backward keeps its
+ *     counter in the caller's workspace.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every
  *     compute entry point only enqueues work and returns; it never
  *     synchronises.  Results are ready when the stream reaches them.
