@@ -78,37 +78,45 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
 
 // The same merge with at most MAXP partials: every LSE and O load of a row is
 // issued before any arithmetic, so a row costs one trip to memory instead of
-// two (the LSE maxima first, then the weighted sum).
-template <typename OutT, int MAXP>
+// two (the LSE maxima first, then the weighted sum).  Each lane covers
+// 4 * VEC columns: with many rows VEC = 2 (a warp takes two rows at d_v = 128,
+// four at 64), so that each resident warp has twice the bytes in flight and
+// the rows need half as many warps; a few rows keep VEC = 1 (shorter per-lane
+// latency chain, and the warps are not the limit there).
+template <typename OutT, int MAXP, int VEC>
 __global__ void __launch_bounds__(256) lse_merge_few_kernel(const float* __restrict__ o_parts,
                                                             const float* __restrict__ lse_parts,
                                                             int P, long long rows, int d_v,
                                                             OutT* __restrict__ out,
                                                             float* __restrict__ lse_out) {
-  const int lanes_per_row = d_v >> 2;
+  const int lanes_per_row = d_v / (4 * VEC);
   const int rows_per_warp = 32 / lanes_per_row;
   const int lane = threadIdx.x & 31;
   const int sub = lane / lanes_per_row;
-  const int col = (lane % lanes_per_row) * 4;
+  const int col = (lane % lanes_per_row) * 4 * VEC;
   const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const long long part_stride = rows * d_v;
   for (long long r = warp * rows_per_warp + sub; r < rows; r += n_warps * rows_per_warp) {
     float l[MAXP];
-    float4 o[MAXP];
+    float4 o[MAXP][VEC];
     const float* src = o_parts + r * d_v + col;
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
       if (p < P) {
         l[p] = __ldg(lse_parts + p * rows + r);
-        o[p] = __ldcs(reinterpret_cast<const float4*>(src + p * part_stride));
+#pragma unroll
+        for (int h = 0; h < VEC; ++h)
+          o[p][h] = __ldcs(reinterpret_cast<const float4*>(src + p * part_stride + 4 * h));
       }
     }
     float m = -INFINITY;
 #pragma unroll
     for (int p = 0; p < MAXP; ++p)
       if (p < P) m = fmaxf(m, l[p]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc[VEC];
+#pragma unroll
+    for (int h = 0; h < VEC; ++h) acc[h] = make_float4(0.f, 0.f, 0.f, 0.f);
     float w_sum = 0.f;
     if (m != -INFINITY) {
 #pragma unroll
@@ -116,16 +124,23 @@ __global__ void __launch_bounds__(256) lse_merge_few_kernel(const float* __restr
         if (p < P) {
           const float w = (l[p] == -INFINITY) ? 0.f : expf(l[p] - m);
           w_sum += w;
-          acc.x = fmaf(w, o[p].x, acc.x);
-          acc.y = fmaf(w, o[p].y, acc.y);
-          acc.z = fmaf(w, o[p].z, acc.z);
-          acc.w = fmaf(w, o[p].w, acc.w);
+#pragma unroll
+          for (int h = 0; h < VEC; ++h) {
+            acc[h].x = fmaf(w, o[p][h].x, acc[h].x);
+            acc[h].y = fmaf(w, o[p][h].y, acc[h].y);
+            acc[h].z = fmaf(w, o[p][h].z, acc[h].z);
+            acc[h].w = fmaf(w, o[p][h].w, acc[h].w);
+          }
         }
       }
       const float inv = 1.f / w_sum;
-      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+#pragma unroll
+      for (int h = 0; h < VEC; ++h) {
+        acc[h].x *= inv; acc[h].y *= inv; acc[h].z *= inv; acc[h].w *= inv;
+      }
     }
-    store4<OutT>(out + r * d_v + col, acc);
+#pragma unroll
+    for (int h = 0; h < VEC; ++h) store4<OutT>(out + r * d_v + col + 4 * h, acc[h]);
     if (lse_out != nullptr && col == 0) {
       lse_out[r] = (m == -INFINITY) ? -INFINITY : m + logf(w_sum);
     }
@@ -224,19 +239,29 @@ int launch_lse_merge(const float* o_parts, const float* lse_parts, int P, long l
       lse_merge_splitp_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
           o_parts, lse_parts, P, rows, d_v, static_cast<__nv_bfloat16*>(out), lse);
   } else {
-    const int rows_per_cta = (threads / 32) * rows_per_warp;
+    // P <= 4 with more rows than one row per resident warp covers: two float4
+    // per lane, twice the rows per warp
+    const bool wide = P <= 4 && warps_needed > static_cast<long long>(num_sms) * 32;
+    const int rows_per_cta = (threads / 32) * (wide ? 2 * rows_per_warp : rows_per_warp);
     long long want = (rows + rows_per_cta - 1) / rows_per_cta;
     long long cap = static_cast<long long>(num_sms) * 8;   // 8 resident CTAs / SM
     int grid = static_cast<int>(want < cap ? want : cap);
     if (grid < 1) grid = 1;
-    // Up to four partials fit in registers at 48 per thread; more would cut the
-    // resident warps (8 partials: 70 registers, 24 warps per SM instead of 64)
-    // and lose more than the single round trip gains, so those loop.
-    if (P <= 4 && out_dtype == RA_F32) {
-      lse_merge_few_kernel<float, 4><<<grid, threads, 0, stream>>>(
+    // Up to four partials fit in registers (48 per thread with one float4 a
+    // lane, 64 with two); more would cut the resident warps (8 partials: 70
+    // registers, 24 warps per SM instead of 64) and lose more than the single
+    // round trip gains, so those loop.
+    if (P <= 4 && wide && out_dtype == RA_F32) {
+      lse_merge_few_kernel<float, 4, 2><<<grid, threads, 0, stream>>>(
+          o_parts, lse_parts, P, rows, d_v, static_cast<float*>(out), lse);
+    } else if (P <= 4 && wide) {
+      lse_merge_few_kernel<__nv_bfloat16, 4, 2><<<grid, threads, 0, stream>>>(
+          o_parts, lse_parts, P, rows, d_v, static_cast<__nv_bfloat16*>(out), lse);
+    } else if (P <= 4 && out_dtype == RA_F32) {
+      lse_merge_few_kernel<float, 4, 1><<<grid, threads, 0, stream>>>(
           o_parts, lse_parts, P, rows, d_v, static_cast<float*>(out), lse);
     } else if (P <= 4) {
-      lse_merge_few_kernel<__nv_bfloat16, 4><<<grid, threads, 0, stream>>>(
+      lse_merge_few_kernel<__nv_bfloat16, 4, 1><<<grid, threads, 0, stream>>>(
           o_parts, lse_parts, P, rows, d_v, static_cast<__nv_bfloat16*>(out), lse);
     } else if (out_dtype == RA_F32) {
       lse_merge_kernel<float><<<grid, threads, 0, stream>>>(o_parts, lse_parts, P, rows, d_v,
