@@ -17,13 +17,18 @@ void note_launch();
 // Releases the copy streams and events of ra_ring_forward_host (ra_shutdown).
 void release_host_call_state();
 
-// Per-device state: SM count, status word address, wait bound.
+// Per-device state: SM count, status word address, wait bound, and the
+// ring of work-item counters the forward launches take slots of.
+constexpr int kItemCounterSlots = 1024;
 struct DeviceInfo {
   int device;
   int num_sms;
   int max_smem_optin;
+  unsigned int* item_counters;  // [kItemCounterSlots] device memory (module global)
   DevCtx ctx;
 };
+// The next slot of the device's counter ring, zeroed on `stream`.
+int next_item_counter(const DeviceInfo& dev, cudaStream_t stream, unsigned int** out);
 int device_info(DeviceInfo* out);
 
 int launch_lse_merge(const float* o_parts, const float* lse_parts, int P, long long rows, int d_v,

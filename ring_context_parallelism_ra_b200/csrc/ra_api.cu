@@ -12,12 +12,18 @@
 
 // One status word per device (module globals are instantiated per device).
 __device__ int g_ra_status_word;
+// Work-item counters of the forward launches: each launch takes the next slot
+// and zeroes it on its stream before the kernel, so launches that run at the
+// same time on different streams use different slots as long as fewer than
+// kItemCounterSlots are in flight.
+__device__ unsigned int g_ra_item_counters[ra::kItemCounterSlots];
 
 namespace ra {
 
 namespace {
 
 std::atomic<unsigned long long> g_launches{0};
+std::atomic<unsigned int> g_counter_next{0};
 std::atomic<unsigned long long> g_wait_ns{2000000000ull};
 
 constexpr int kMaxDevices = 64;
@@ -146,6 +152,13 @@ __global__ void wait_timeout_kernel(DevCtx ctx) {
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+int next_item_counter(const DeviceInfo& dev, cudaStream_t stream, unsigned int** out) {
+  unsigned int* c = dev.item_counters + (g_counter_next.fetch_add(1) % kItemCounterSlots);
+  if (cudaMemsetAsync(c, 0, sizeof(unsigned int), stream) != cudaSuccess) return RA_ERR_CUDA;
+  *out = c;
+  return RA_OK;
+}
+
 int device_info(DeviceInfo* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RA_ERR_CUDA;
@@ -160,6 +173,8 @@ int device_info(DeviceInfo* out) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_ra_status_word) != cudaSuccess) return RA_ERR_CUDA;
     d.ctx.status = static_cast<int*>(p);
+    if (cudaGetSymbolAddress(&p, g_ra_item_counters) != cudaSuccess) return RA_ERR_CUDA;
+    d.item_counters = static_cast<unsigned int*>(p);
     g_dev[dev] = d;
     g_dev_ready[dev] = true;
   }

@@ -43,9 +43,6 @@
 // max keeps p <= 256; the final division by l makes the result exact).
 #include <cuda.h>
 
-#include <atomic>
-#include <mutex>
-
 #include "block_class.cuh"
 #include "common.cuh"
 #include "item_queue.cuh"
@@ -773,37 +770,6 @@ int dispatch(int dqk, int dv, const CUtensorMap& tq, const CUtensorMap& tk, cons
 
 }  // namespace
 
-namespace {
-
-// Work-item counters of the forward launches: a ring of slots in device
-// memory (one array per device); each launch takes the next slot and zeroes
-// it on its stream before the kernel.  Launches that run at the same time on
-// different streams use different slots as long as fewer than kCounterSlots
-// are in flight.
-constexpr int kCounterSlots = 1024;
-__device__ unsigned int g_tc_item_counters[kCounterSlots];
-std::mutex g_ctr_mu;
-unsigned int* g_ctr_base[64] = {};
-std::atomic<unsigned int> g_ctr_next{0};
-
-int item_counter_slot(int device, cudaStream_t stream, unsigned int** out) {
-  if (device < 0 || device >= 64) return RA_ERR_CUDA;
-  {
-    std::lock_guard<std::mutex> lock(g_ctr_mu);
-    if (g_ctr_base[device] == nullptr) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_tc_item_counters) != cudaSuccess) return RA_ERR_CUDA;
-      g_ctr_base[device] = static_cast<unsigned int*>(p);
-    }
-  }
-  unsigned int* c = g_ctr_base[device] + (g_ctr_next.fetch_add(1) % kCounterSlots);
-  if (cudaMemsetAsync(c, 0, sizeof(unsigned int), stream) != cudaSuccess) return RA_ERR_CUDA;
-  *out = c;
-  return RA_OK;
-}
-
-}  // namespace
-
 int launch_tc_attention(const void* q, const void* k, const void* v, const ra_shape& s, int P,
                         int q_offset, int k_offset, long long stride, int causal,
                         int striped, float scale, void* out, bool out_f32, float* lse,
@@ -847,7 +813,7 @@ int launch_tc_attention(const void* q, const void* k, const void* v, const ra_sh
   const long long n_kv = static_cast<long long>(s.B) * s.Hkv;
   a.kv_block = static_cast<int>(fit < 1 ? 1 : (fit > n_kv ? n_kv : fit));
   a.ctx = dev.ctx;
-  const int rc = item_counter_slot(dev.device, stream, &a.item_counter);
+  const int rc = next_item_counter(dev, stream, &a.item_counter);
   if (rc != RA_OK) return rc;
   const int grid = a.items < dev.num_sms ? a.items : dev.num_sms;
   return out_f32 ? dispatch<true>(s.d_qk, s.d_v, tq, tk, tv, a, grid, stream)
