@@ -117,3 +117,29 @@ def test_committed_traffic_matches_current_kernel_sources():
     # code; the bench reports them only while the code is unchanged
     assert bench.load_traffic("ring_forward:causal_mha_b1_h8_n8192_d128_P4", bench.TC_FILES)
     assert bench.load_traffic("ring_backward:causal_mha_b1_h8_n8192_d128_P4", bench.BWD_FILES)
+
+
+def test_recap_carries_every_leg_in_a_short_tail():
+    # a line shaped like the GPU arm's: the recap repeats each leg's value and
+    # fraction, and with the decode leg after it the last 1500 characters hold
+    # recap, decode and the decode short-cache latencies
+    def entry(name, value, frac):
+        return {"workload": name, "value": value, "roofline": {"frac": frac, "pad": "x" * 400}}
+    line = {"value": 1100.0, "roofline": {"frac": 0.67}, "config": {"workload": "w5"},
+            "e2e": {"value": 1050.0},
+            "workloads": [entry("w3", 1000.0, 0.61), entry("w2", 900.0, 0.55)],
+            "backward": [entry("w5", 760.0, 0.46), entry("w3", 850.0, 0.52)],
+            "merge": [{"value": 2500.0}, {"value": 6100.0}],
+            "striped": {"ring_speedup_striped_over_contiguous": 1.78},
+            "cpu_baseline": {"value": 0.01, "sample": "y" * 300},
+            "decode_short_cache": {"tokens": 32768, "pad": "z" * 150},
+            "decode": {"value": 6900.0, "pad": "d" * 400}}
+    r = bench.recap(line)
+    assert r["prefill"] == {"w5": [1100.0, 0.67], "w3": [1000.0, 0.61], "w2": [900.0, 0.55]}
+    assert r["backward"] == {"w5": [760.0, 0.46], "w3": [850.0, 0.52]}
+    assert r["e2e_tflops"] == 1050.0 and r["merge_gbs"] == [2500.0, 6100.0]
+    line["recap"] = r
+    for key in ("decode_short_cache", "decode"):
+        line[key] = line.pop(key)
+    tail = json.dumps(line)[-1500:]
+    assert '"recap"' in tail and '"decode"' in tail
